@@ -1,0 +1,383 @@
+"""Benchmark: ReplaySSM decode of a Mamba-2 layer at serving shape.
+
+Workload (one GPU): batch 256, 80 heads, headdim 64, dstate 128, 1 group, bf16
+inputs, fp32 master checkpoint + bf16 output copy, commit interval K = 8, the
+checkpoint seeded by a 512-token eager prefill.  A step is one pass of the
+decode path over the batch: append the step's inputs to the ring, compute the
+outputs by output-only replay, and commit every 8th step.  The checkpoint
+(335 MB bf16 + 671 MB fp32) is larger than L2, so no flush is needed between
+steps.
+
+Prints one JSON line.  `--impl reference` times the fp64 CPU oracle instead
+(the reference arm: there is no runnable reference implementation).
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+B, H, P, N, G, K_COMMIT, CAP, PREFILL = 256, 80, 64, 128, 1, 8, 16, 512
+POOL = 256          # distinct decode steps of inputs kept resident (cycled)
+METRIC = "SSM-layer decode tokens/s at batch 256; achieved HBM GB/s vs B200 peak"
+UNIT = "tokens/s"
+WORKLOAD = "mamba2-decode-b256-h80-p64-n128-bf16copy-K8"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2048)
+    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--impl", default="rs", choices=["rs", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-work", type=float, default=20.0)
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------- clocks ------
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    def __init__(self, index=0, period=0.01):
+        self.samples, self.reasons, self.period = [], set(), period
+        self.stop_ev = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        names = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+                 "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                r = get(self.h)
+                for n, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(n)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self.stop_ev.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ CPU oracle ---
+
+class OracleSample:
+    """A bounded sample of the workload for the fp64 CPU oracle: nseq
+    sequences x all heads, T decode steps per call, state carried across calls."""
+
+    def __init__(self, nseq, T, seed):
+        import numpy as np
+        rng = np.random.default_rng(seed)
+        n = nseq * H
+        self.nseq, self.T = nseq, T
+        self.A = -np.exp(rng.uniform(0, math.log(16), n))
+        self.D = rng.standard_normal(n)
+        self.x = rng.standard_normal((n, T, P))
+        self.dt = np.log1p(np.exp(rng.standard_normal((n, T)) * 0.5 - 3.0))
+        self.B = rng.standard_normal((n, T, N)) / math.sqrt(N)
+        self.C = rng.standard_normal((n, T, N)) / math.sqrt(N)
+        self.h = rng.standard_normal((n, P, N)) * 0.1
+
+    def run(self, cores):
+        import oracle
+        t0 = time.perf_counter()
+        oracle.mamba2_eager_batch(self.A, self.D, self.x, self.dt, self.B, self.C, h=self.h,
+                                  nthreads=cores)
+        return time.perf_counter() - t0
+
+
+def cpu_oracle_rate(cpu_work_s, nseq=32, T=8, seed=0):
+    """Times the oracle on about `cpu_work_s` seconds of CPU work (wall time x
+    threads).  Returns (tokens/s, threads, sample text)."""
+    cores = os.cpu_count() or 1
+    s = OracleSample(nseq, T, seed)
+    s.run(cores)                                   # warm the pages
+    target = max(0.5, cpu_work_s / cores)
+    el, reps = 0.0, 0
+    while el < target:
+        el += s.run(cores)
+        reps += 1
+    return nseq * T * reps / el, cores, (
+        f"{reps} x ({nseq} sequences x {H} heads x {T} decode steps) of the fp64 eager "
+        f"recurrence ({P}x{N} state per head), {el:.2f} s wall on {cores} threads")
+
+
+def reference_arm(args, rank):
+    if rank != 0:
+        return
+    cores = os.cpu_count() or 1
+    s = OracleSample(4, 4, 0)
+    s.run(cores)
+    for _ in range(args.warmup):
+        s.run(cores)
+    el = sum(s.run(cores) for _ in range(args.steps))
+    value = s.nseq * s.T * args.steps / el
+    sample = (f"per step {s.nseq} sequences x {H} heads x {s.T} decode steps of the fp64 eager "
+              f"recurrence; {args.steps} timed steps, {el:.2f} s wall on {cores} threads")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * B / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "global_batch": B,
+                                            "parallelism": "none (CPU oracle)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------- GPU arm -----
+
+def gpu_arm(args, rank, world):
+    import torch
+    import torch.distributed as dist
+
+    import rs_decode_outputs_b200 as rs
+    from rs_decode_outputs_b200 import inputs as gen
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    seed = 1 + 1000 * rank
+
+    A, D, dtb = gen.mamba2_params(H, seed, dev)
+    src = gen.Mamba2Stream(B, H, P, N, G, torch.bfloat16, dtb, seed + 10_000, dev)
+    cfg = rs.make_config(rs.RS_MAMBA2, B, H, P, N, G, cap=CAP, npos_max=1, in_dtype=rs.RS_BF16,
+                         copy_dtype=rs.RS_BF16, out_dtype=rs.RS_BF16)
+    sess = rs.ReplaySSM(cfg, A=A, D=D, device=dev)
+
+    # prefill: 512 eager fp32 steps on a state tensor, then load it as the checkpoint
+    state = torch.zeros(B, H, P, N, device=dev)
+    ypre = torch.empty(1, B, H, P, device=dev, dtype=torch.bfloat16)
+    for c in range(PREFILL // 64):
+        chunk = src.next(64)
+        for t in range(64):
+            sess.eager_step(state, rs.RS_F32, {k: v[t:t + 1] for k, v in chunk.items()}, 1, ypre)
+    sess.load_checkpoint(state)
+    del state
+
+    pool = src.next(POOL)
+    steps_in = [{k: v[t:t + 1] for k, v in pool.items()} for t in range(POOL)]
+    y = sess.new_out()
+    h = sess.handle
+
+    def step(i, ev=None):
+        rs.rs_append(h, rs.make_inputs(steps_in[i % POOL]), 1)
+        if ev is not None:
+            ev[0].record(stream)
+        rs.rs_decode_outputs(h, y)
+        if ev is not None:
+            ev[1].record(stream)
+        if (i + 1) % K_COMMIT == 0:
+            if ev is not None:
+                ev[2].record(stream)
+            rs.rs_commit(h, K_COMMIT)
+            if ev is not None:
+                ev[3].record(stream)
+
+    i = 0
+    for _ in range(args.warmup):
+        step(i)
+        i += 1
+    # align the timed region to commit boundaries so every K-th step commits
+    while i % K_COMMIT:
+        step(i)
+        i += 1
+
+    # pass 1: whole-step throughput (no per-kernel events)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = rs.rs_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step(i)
+            i += 1
+        e1.record(stream)
+        torch.cuda.synchronize()
+    launches = rs.rs_launch_count() - n0
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+
+    # pass 2: per-kernel durations (events around each launch) for the roofline
+    nk = min(args.steps, 512)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nk)]
+    torch.cuda.synchronize()
+    for j in range(nk):
+        step(i, evs[j])
+        i += 1
+    torch.cuda.synchronize()
+    dec_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    com_ms = [e[2].elapsed_time(e[3]) for e, j in zip(evs, range(nk)) if (i - nk + j + 1) % K_COMMIT == 0]
+
+    # eager read-modify-write baseline on the same shape (fp32 state and bf16 state)
+    eager = {}
+    for name, sdt, tdt, ebytes in (("fp32", rs.RS_F32, torch.float32, 4), ("bf16", rs.RS_BF16, torch.bfloat16, 2)):
+        st = torch.zeros(B, H, P, N, device=dev, dtype=tdt)
+        ye = torch.empty(1, B, H, P, device=dev, dtype=torch.bfloat16)
+        for j in range(8):
+            sess.eager_step(st, sdt, steps_in[j], 1, ye)
+        ne = min(args.steps, 256)
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for j in range(ne):
+            rs.rs_eager_step(h, st, sdt, rs.make_inputs(steps_in[j % POOL]), 1, ye)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        ems = a0.elapsed_time(a1) / ne
+        eager[name] = {"tokens_per_s": B / (ems * 1e-3), "ms_per_step": ems,
+                       "state_bytes_per_token": 2 * ebytes * H * P * N,
+                       "achieved_gbs": 2 * ebytes * B * H * P * N / (ems * 1e-3) / 1e9}
+        del st
+
+    # end to end: inputs from pinned host memory every step, outputs read back
+    ne2e = min(args.steps, 256)
+    host_in = [{k: v.cpu().pin_memory() for k, v in steps_in[j].items()} for j in range(min(POOL, ne2e))]
+    dev_in = {k: torch.empty_like(v) for k, v in steps_in[0].items()}
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host_in[0].values())
+    d2h = y.numel() * y.element_size()
+    torch.cuda.synchronize()
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b0.record(stream)
+    for j in range(ne2e):
+        for k, v in host_in[j % len(host_in)].items():
+            dev_in[k].copy_(v, non_blocking=True)
+        rs.rs_append(h, rs.make_inputs(dev_in), 1)
+        rs.rs_decode_outputs(h, y)
+        if (i + 1) % K_COMMIT == 0:
+            rs.rs_commit(h, K_COMMIT)
+        i += 1
+        y_host.copy_(y, non_blocking=True)
+    b1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = b0.elapsed_time(b1) / ne2e
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    status, flags = sess.get_error()
+    if status != rs.RS_OK:
+        raise RuntimeError(f"device error flags set: {set(flags.tolist())}")
+
+    if rank != 0:
+        return
+    hbm, peak_kind = peaks()
+    copy_bytes = B * H * P * N * 2
+    y_bytes = B * H * P * 2
+    dec_avg = statistics.mean(dec_ms)
+    achieved = (copy_bytes + y_bytes) / (dec_avg * 1e-3) / 1e9
+    com_avg = statistics.mean(com_ms) if com_ms else float("nan")
+    commit_bytes = B * H * P * N * (4 + 4 + 2)
+    step_ms = ms / args.steps
+    value = world * B * args.steps / (ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; Mamba-2 serving-shape distributions)",
+        "config": {"workload": WORKLOAD, "global_batch": B * world, "batch_per_gpu": B,
+                   "nheads": H, "headdim": P, "dstate": N, "ngroups": G, "commit_interval": K_COMMIT,
+                   "ring_cap": CAP, "prefill_tokens": PREFILL, "checkpoint": "fp32 master + bf16 copy",
+                   "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
+                   "l2": "inputs larger than L2 (checkpoint copy 335 MB per step), no flush"},
+        "roofline": {"bound": "hbm", "kernel": "m2_outputs_kernel (output-only replay)",
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": None, "peak_source": peak_kind,
+                     "algorithmic_bytes_per_launch": copy_bytes + y_bytes,
+                     "avg_launch_us": dec_avg * 1e3},
+        "kernels": {"decode_us": dec_avg * 1e3, "commit_us": com_avg * 1e3,
+                    "commit_gbs": commit_bytes / (com_avg * 1e-3) / 1e9 if com_ms else None,
+                    "step_state_bytes_per_token": H * P * N * (2 + 10 / K_COMMIT),
+                    "step_achieved_gbs": B * H * P * N * (2 + 10 / K_COMMIT) / (step_ms * 1e-3) / 1e9},
+        "eager": eager,
+        "e2e": {"value": world * B / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    if not args.no_cpu_baseline:
+        v, cores, sample = cpu_oracle_rate(args.cpu_work)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        reference_arm(args, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        gpu_arm(args, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

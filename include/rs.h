@@ -1,0 +1,221 @@
+/*
+ * rs.h -- C interface of the ReplaySSM decode library (librs_b200.so).
+ *
+ * ReplaySSM ("ReplaySSM: Cache SSM Inputs, Not State", Abstract) represents the
+ * recurrent state of each sequence of a Mamba-2 or Gated DeltaNet layer as a
+ * read-only checkpoint plus a buffer of the SSM inputs seen since that
+ * checkpoint.  Each decode step's output is computed from the checkpoint and
+ * the buffer without writing state; the checkpoint is rewritten only when the
+ * caller commits; speculative tokens are rejected by moving the buffer's tail
+ * pointer; a high-precision master checkpoint serves the updates while a
+ * low-precision copy serves the outputs.
+ *
+ * Recurrences (the pages give none; the standard published forms are used):
+ *   Mamba-2:  h_t = exp(dt_t A) h_{t-1} + dt_t x_t B_t^T,   y_t = h_t C_t + D x_t
+ *             state tile per (sequence, head): [P][N], row p, column n
+ *   GDN:      S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *             o_t = gdn_scale * S_t q_t
+ *             state tile per (sequence, head): [dv][dk], row r, column c
+ *
+ * Conventions for every call
+ *   - All data pointers are DEVICE pointers unless a parameter says "host".
+ *   - Every call is asynchronous on the given stream (a cudaStream_t passed as
+ *     void*; NULL means the legacy default stream) unless it says "synchronises".
+ *   - The library never allocates device memory.  The caller allocates one
+ *     workspace of rs_workspace_size() bytes (256-byte aligned) that holds the
+ *     checkpoints, the input ring and the pointers; it must outlive the handle.
+ *   - Host-checkable problems (NULL pointers, bad shapes, T > cap, npos out of
+ *     range) return an error and launch nothing.  Data-dependent problems found
+ *     on the device (ring overflow, rollback past the checkpoint, too few
+ *     buffered entries) leave that sequence's pointers unchanged, write zeros for
+ *     its outputs and set a sticky bit in its error word (rs_get_error).  No call
+ *     traps or spins without a bound on the device.
+ *   - Dense layouts, row-major, no padding:  B = batch, H = nheads,
+ *     R = rows of a state tile (Mamba-2 P = headdim, GDN dv = headdim),
+ *     Cc = columns (Mamba-2 N = dstate, GDN dk = dstate), G = ngroups.
+ */
+#ifndef RS_H
+#define RS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct rs_ctx *rs_handle;
+typedef void *rs_stream; /* cudaStream_t */
+
+typedef enum {
+    RS_OK = 0,
+    RS_ERR_ARG = -1,          /* invalid argument or configuration */
+    RS_ERR_CAPACITY = -2,     /* T or npos larger than the ring allows */
+    RS_ERR_CUDA = -4,         /* a CUDA runtime call failed (rs_last_cuda_error) */
+    RS_ERR_WORKSPACE = -5,    /* workspace NULL, misaligned or too small */
+    RS_ERR_DEVICE_FLAG = -6,  /* rs_get_error: some sequence has a sticky error bit */
+    RS_ERR_UNSUPPORTED = -8   /* valid but unsupported shape / dtype combination */
+} rs_status;
+
+typedef enum { RS_MAMBA2 = 0, RS_GDN = 1 } rs_kind;
+
+typedef enum {
+    RS_NONE = 0,  /* no low-precision copy: outputs read the fp32 master */
+    RS_F32 = 1,
+    RS_BF16 = 2,  /* bfloat16, round to nearest even */
+    RS_E4M3 = 3   /* OCP FP8 E4M3 (fn), RNE, satfinite, one fp32 scale per tile */
+} rs_dtype;
+
+/* Per-sequence sticky device error bits (rs_get_error). */
+enum {
+    RS_SEQ_ERR_OVERFLOW = 1u,  /* rs_append: len + T > cap; nothing written      */
+    RS_SEQ_ERR_ROLLBACK = 2u,  /* rs_rollback / rs_eager_accept: k outside range */
+    RS_SEQ_ERR_EMPTY = 4u,     /* outputs asked for with len < npos (or len 0)   */
+    RS_SEQ_ERR_TIMEOUT = 8u    /* a bounded on-device wait gave up               */
+};
+
+typedef struct {
+    int32_t kind;        /* rs_kind */
+    int32_t batch;       /* B >= 1 sequences */
+    int32_t nheads;      /* H >= 1 */
+    int32_t headdim;     /* R: Mamba-2 P, GDN dv; 1..256 */
+    int32_t dstate;      /* Cc: Mamba-2 N, GDN dk; one of 16, 32, 64, 128, 256 */
+    int32_t ngroups;     /* Mamba-2 G, divides H (head h uses group h / (H/G)); GDN: 1 */
+    int32_t cap;         /* ring slots per sequence: power of two, 1..256 */
+    int32_t npos_max;    /* largest npos of rs_verify_outputs / rs_eager_verify: 1..8 */
+    int32_t in_dtype;    /* RS_F32 or RS_BF16: x, B, C (Mamba-2) / q, k, v (GDN) */
+    int32_t copy_dtype;  /* RS_NONE, RS_BF16 or RS_E4M3: the output copy */
+    int32_t out_dtype;   /* RS_F32 or RS_BF16: y / o */
+    int32_t shared_lowp; /* 1: no fp32 master; the low-precision copy serves both
+                            outputs and updates (the comparison arm of step 5) */
+    float gdn_scale;     /* GDN output scale; 0 is taken as 1 */
+} rs_config;
+
+/* Step inputs.  Mamba-2 uses x, dt, B, C; GDN uses q, k, v, alpha, beta.
+ * dt, alpha, beta are fp32; the others are in_dtype.  Shapes for T steps:
+ *   x [T][B][H][P]   dt [T][B][H]   B, C [T][B][G][N]      (dt after softplus)
+ *   q, k [T][B][H][dk]   v [T][B][H][dv]   alpha, beta [T][B][H]              */
+typedef struct {
+    const void *x;
+    const float *dt;
+    const void *B;
+    const void *C;
+    const void *q;
+    const void *k;
+    const void *v;
+    const float *alpha;
+    const float *beta;
+} rs_inputs;
+
+/* Byte offsets of the regions of a workspace (each 256-byte aligned; a region a
+ * configuration does not use has size 0).  Tests and tools use this to view the
+ * checkpoints and pointers; kernels get the same offsets. */
+typedef struct {
+    size_t master, master_bytes;   /* fp32 [B][H][R][Cc]          (not with shared_lowp) */
+    size_t copy, copy_bytes;       /* copy_dtype [B][H][R][Cc]    (not with RS_NONE)     */
+    size_t scale, scale_bytes;     /* fp32 [B][H]                 (RS_E4M3 only)         */
+    size_t ring_a, ring_a_bytes;   /* Mamba-2 x [B][cap][H][P]   | GDN q [B][cap][H][dk] */
+    size_t ring_b, ring_b_bytes;   /* Mamba-2 dt [B][cap][H] f32 | GDN k [B][cap][H][dk] */
+    size_t ring_c, ring_c_bytes;   /* Mamba-2 B [B][cap][G][N]   | GDN v [B][cap][H][dv] */
+    size_t ring_d, ring_d_bytes;   /* Mamba-2 C [B][cap][G][N]   | GDN alpha [B][cap][H] */
+    size_t ring_e, ring_e_bytes;   /* (unused for Mamba-2)       | GDN beta [B][cap][H]  */
+    size_t head, tail, err, arrive;/* int32 / int32 / uint32 / uint32, each [B]          */
+    size_t total;
+} rs_layout;
+
+/* Workspace size and layout for a configuration.  Pure host computation; needs
+ * no GPU.  Returns RS_ERR_ARG / RS_ERR_UNSUPPORTED for a bad configuration. */
+rs_status rs_workspace_size(const rs_config *cfg, size_t *bytes);
+rs_status rs_workspace_layout(const rs_config *cfg, rs_layout *layout);
+
+/* Create a handle over a caller-allocated workspace.  A and D (Mamba-2 only,
+ * fp32 [H], device; D may be NULL for 0) are copied into the handle's view by
+ * pointer: they must stay valid for the handle's lifetime.  Zeroes the
+ * workspace on `stream` (checkpoint = 0, head = tail = 0, no errors, fp8
+ * scales = 1).  The handle itself is host memory owned by the library. */
+rs_status rs_create(const rs_config *cfg, void *workspace, size_t workspace_bytes,
+                    const float *A, const float *D, rs_stream stream, rs_handle *out);
+rs_status rs_destroy(rs_handle h);
+
+/* Replace every checkpoint by `state` (fp32 [B][H][R][Cc], device) -- e.g. the
+ * state after a prompt -- derive the low-precision copy from it, and empty the
+ * buffer (head = tail = 0); error words are cleared.  With shared_lowp the
+ * state is quantised straight into the copy. */
+rs_status rs_load_checkpoint(rs_handle h, const float *state, rs_stream stream);
+
+/* Append T >= 1 inputs per sequence at the tail of its ring ("ReplaySSM for
+ * hybrid SSM-Transformer stacks", How ReplaySSM works, step 2: append the new
+ * SSM input to the buffer).  A sequence whose len + T would exceed cap gets
+ * RS_SEQ_ERR_OVERFLOW and is left unchanged.  T > cap returns RS_ERR_CAPACITY. */
+rs_status rs_append(rs_handle h, const rs_inputs *in, int T, rs_stream stream);
+
+/* Output of the newest buffered input of every sequence, computed from the
+ * checkpoint and the buffer without writing any state (Abstract: output
+ * computation separated from checkpoint updates; How ReplaySSM works, step 2:
+ * no intermediate states are materialised).  Reads the low-precision copy
+ * (the fp32 master when copy_dtype is RS_NONE).  y: out_dtype [B][H][R].
+ * A sequence with an empty buffer gets zeros and RS_SEQ_ERR_EMPTY. */
+rs_status rs_decode_outputs(rs_handle h, void *y, rs_stream stream);
+
+/* Commit (How ReplaySSM works, step 3): for every sequence with
+ * len >= max(min_len, 1) and, when mask is not NULL, mask[b] != 0 (int32 [B],
+ * device), apply the recurrence from the fp32 master across the buffered
+ * inputs, write the new master and re-derive the copy from it (step 5: the
+ * master is never derived from the copy), then empty the buffer (head = tail).
+ * With shared_lowp the fold starts from the dequantised copy instead. */
+rs_status rs_commit(rs_handle h, int min_len, const int32_t *mask, rs_stream stream);
+
+/* Output-only verification (Abstract; How ReplaySSM works, step 4): outputs at
+ * the newest npos buffered positions of every sequence from one pass over the
+ * checkpoint, without materialising intermediate states.  1 <= npos <= npos_max.
+ * y: out_dtype [npos][B][H][R], position 0 the oldest of the npos.  A sequence
+ * with len < npos gets zeros and RS_SEQ_ERR_EMPTY. */
+rs_status rs_verify_outputs(rs_handle h, int npos, void *y, rs_stream stream);
+
+/* Pointer-only rollback (How ReplaySSM works, step 4: move the buffer tail back
+ * by k entries; the checkpoint never changes).  k: int32 [B], device.  A
+ * sequence with k outside [0, len] gets RS_SEQ_ERR_ROLLBACK and is unchanged. */
+rs_status rs_rollback(rs_handle h, const int32_t *k, rs_stream stream);
+
+/* Eager read-modify-write baseline ("What ReplaySSM is solving": read the whole
+ * state, update it, write it back, every step).  Applies T >= 1 steps of the
+ * recurrence to `state` (state_dtype RS_F32 or RS_BF16, [B][H][R][Cc], device,
+ * caller-owned, independent of the handle's checkpoints) and writes the output
+ * of every step, y: out_dtype [T][B][H][R].  Uses the handle's shapes, A, D,
+ * gdn_scale.  Also serves as the prompt (prefill) pass before rs_load_checkpoint. */
+rs_status rs_eager_step(rs_handle h, void *state, int state_dtype, const rs_inputs *in, int T,
+                        void *y, rs_stream stream);
+
+/* Eager speculative baseline: for npos positions, read the state once from
+ * slot cur[b] of `slots` (state_dtype [npos_max + 1][B][H][R][Cc]), apply the
+ * npos updates in order, write each intermediate state to slot
+ * (cur[b] + 1 + p) mod (npos_max + 1) and each output to y [npos][B][H][R].
+ * rs_eager_accept then makes the state after keep[b] positions current:
+ * cur[b] = (cur[b] + keep[b]) mod (npos_max + 1); keep outside [0, npos_max]
+ * sets RS_SEQ_ERR_ROLLBACK.  cur, keep: int32 [B], device. */
+rs_status rs_eager_verify(rs_handle h, void *slots, int state_dtype, const int32_t *cur,
+                          const rs_inputs *in, int npos, void *y, rs_stream stream);
+rs_status rs_eager_accept(rs_handle h, int32_t *cur, const int32_t *keep, rs_stream stream);
+
+/* Synchronises `stream`, then copies the per-sequence error words to
+ * seq_flags_host (uint32 [B], host, may be NULL) and their OR to *any_host
+ * (may be NULL).  Returns RS_ERR_DEVICE_FLAG when any bit is set. */
+rs_status rs_get_error(rs_handle h, uint32_t *seq_flags_host, uint32_t *any_host,
+                       rs_stream stream);
+rs_status rs_clear_error(rs_handle h, rs_stream stream);
+
+/* Synchronises `stream`, then copies head / tail (int32 [B] each, host; either
+ * may be NULL).  head is the position of the checkpoint, tail one past the
+ * newest buffered input; both only grow except that rollback lowers tail. */
+rs_status rs_read_ptrs(rs_handle h, int32_t *head_host, int32_t *tail_host, rs_stream stream);
+
+/* Diagnostics. */
+const char *rs_status_string(int status);
+const char *rs_last_cuda_error(void);     /* text of the last failing CUDA call */
+uint64_t rs_launch_count(void);           /* kernels launched by this library so far */
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RS_H */

@@ -1,0 +1,155 @@
+// Ring-buffer and checkpoint kernels shared by both layer kinds: append,
+// pointer-only rollback, checkpoint load (master + derived copy), workspace
+// initialisation and the eager baseline's slot selection.
+#include "regtile.cuh"
+#include "launch.h"
+
+namespace rs {
+
+// Cooperative copy of nbytes (a multiple of 2) between global buffers, with
+// 16-byte moves when both ends are 16-byte aligned.
+__device__ __forceinline__ void copy_coop(void *dst, const void *src, size_t nbytes) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src);
+    if ((a & 15) == 0 && (nbytes & 15) == 0) {
+        for (size_t i = threadIdx.x; i < nbytes / 16; i += blockDim.x)
+            static_cast<uint4 *>(dst)[i] = static_cast<const uint4 *>(src)[i];
+    } else if ((a & 3) == 0 && (nbytes & 3) == 0) {
+        for (size_t i = threadIdx.x; i < nbytes / 4; i += blockDim.x)
+            static_cast<uint32_t *>(dst)[i] = static_cast<const uint32_t *>(src)[i];
+    } else {
+        for (size_t i = threadIdx.x; i < nbytes / 2; i += blockDim.x)
+            static_cast<uint16_t *>(dst)[i] = static_cast<const uint16_t *>(src)[i];
+    }
+}
+
+// ----------------------------------------------------------------- append --
+// One CTA per sequence ("ReplaySSM for hybrid SSM-Transformer stacks", How
+// ReplaySSM works, step 2: append the step's SSM input to the buffer).  Writes
+// slots tail .. tail+T-1 (mod cap), then advances tail.  Refuses, with a sticky
+// error bit, when the buffer would hold more than cap entries.
+__global__ void __launch_bounds__(256) append_kernel(const Params p, rs_inputs in, int T, int kind) {
+    const int b = blockIdx.x;
+    const int head = p.head[b], tail = p.tail[b];
+    if (tail - head + T > p.cap || tail - head < 0) {
+        if (threadIdx.x == 0) atomicOr(&p.err[b], RS_SEQ_ERR_OVERFLOW);
+        return;
+    }
+    const int H = p.H, R = p.R, CC = p.CC, Bn = p.B;
+    const size_t ib = p.in_dtype == RS_BF16 ? 2 : 4;
+    for (int t = 0; t < T; ++t) {
+        const size_t row = (size_t)b * p.cap + ((tail + t) & p.cap_mask);   // ring row of this entry
+        const size_t src = (size_t)t * Bn + b;                              // input row [t][b]
+        if (kind == RS_MAMBA2) {
+            const size_t nx = (size_t)H * R, nbc = (size_t)p.G * CC;
+            copy_coop(static_cast<char *>(p.ra) + row * nx * ib, static_cast<const char *>(in.x) + src * nx * ib, nx * ib);
+            copy_coop(static_cast<float *>(p.rb) + row * H, in.dt + src * H, (size_t)H * 4);
+            copy_coop(static_cast<char *>(p.rc) + row * nbc * ib, static_cast<const char *>(in.B) + src * nbc * ib, nbc * ib);
+            copy_coop(static_cast<char *>(p.rd) + row * nbc * ib, static_cast<const char *>(in.C) + src * nbc * ib, nbc * ib);
+        } else {
+            const size_t nk = (size_t)H * CC, nv = (size_t)H * R;
+            copy_coop(static_cast<char *>(p.ra) + row * nk * ib, static_cast<const char *>(in.q) + src * nk * ib, nk * ib);
+            copy_coop(static_cast<char *>(p.rb) + row * nk * ib, static_cast<const char *>(in.k) + src * nk * ib, nk * ib);
+            copy_coop(static_cast<char *>(p.rc) + row * nv * ib, static_cast<const char *>(in.v) + src * nv * ib, nv * ib);
+            copy_coop(static_cast<float *>(p.rd) + row * H, in.alpha + src * H, (size_t)H * 4);
+            copy_coop(static_cast<float *>(p.re) + row * H, in.beta + src * H, (size_t)H * 4);
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) p.tail[b] = tail + T;
+}
+
+cudaError_t launch_append(const Params &p, const rs_inputs &in, int T, cudaStream_t st) {
+    append_kernel<<<p.B, 256, 0, st>>>(p, in, T, p.kind);
+    return cudaGetLastError();
+}
+
+// --------------------------------------------------------------- rollback --
+// How ReplaySSM works, step 4: rejecting the last k tokens moves the tail back
+// by k; the checkpoint is not touched.  Integer-only, one thread per sequence.
+__global__ void rollback_kernel(const Params p, const int32_t *__restrict__ k) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= p.B) return;
+    const int kb = k[b];
+    const int len = p.tail[b] - p.head[b];
+    if (kb < 0 || kb > len) atomicOr(&p.err[b], RS_SEQ_ERR_ROLLBACK);
+    else p.tail[b] -= kb;
+}
+
+cudaError_t launch_rollback(const Params &p, const int32_t *k, cudaStream_t st) {
+    rollback_kernel<<<(p.B + 255) / 256, 256, 0, st>>>(p, k);
+    return cudaGetLastError();
+}
+
+// Eager baseline's "rollback": the state after keep[b] accepted positions
+// becomes current, by index.
+__global__ void eager_accept_kernel(const Params p, int32_t *cur, const int32_t *__restrict__ keep,
+                                    int nslots) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= p.B) return;
+    const int kb = keep[b];
+    if (kb < 0 || kb > nslots - 1) atomicOr(&p.err[b], RS_SEQ_ERR_ROLLBACK);
+    else cur[b] = (cur[b] + kb) % nslots;
+}
+
+cudaError_t launch_eager_accept(const Params &p, int32_t *cur, const int32_t *keep, int nslots,
+                                cudaStream_t st) {
+    eager_accept_kernel<<<(p.B + 255) / 256, 256, 0, st>>>(p, cur, keep, nslots);
+    return cudaGetLastError();
+}
+
+// --------------------------------------------------------- load checkpoint --
+// Replace the checkpoint by an fp32 state: write the master and derive the
+// copy from it (How ReplaySSM works, step 5: the copy is always derived from
+// the high-precision checkpoint); the buffer becomes empty.
+template <int CC, int NPASS>
+__global__ void __launch_bounds__(kTileThreads) load_checkpoint_kernel(const Params p, const float *state) {
+    __shared__ float red[kTileThreads / 32];
+    const int tile = blockIdx.x;
+    RegTile<CC, NPASS> t;
+    t.init(p.R);
+    t.load_f32(state + (size_t)tile * p.R * CC);
+    if (!p.shared_lowp) t.store_f32(p.master + (size_t)tile * p.R * CC);
+    if (p.copy_dtype != RS_NONE) store_tile(t, p.copy, tile, p.copy_dtype, p.scale, red);
+    if (tile % p.H == 0 && threadIdx.x == 0) {
+        const int b = tile / p.H;
+        p.head[b] = 0;
+        p.tail[b] = 0;
+        p.err[b] = 0u;
+        p.arrive[b] = 0u;
+    }
+}
+
+template <int CC, int NPASS>
+static cudaError_t launch_load_t(const Params &p, const float *state, cudaStream_t st) {
+    load_checkpoint_kernel<CC, NPASS><<<p.B * p.H, kTileThreads, 0, st>>>(p, state);
+    return cudaGetLastError();
+}
+
+template <int CC>
+static cudaError_t launch_load_cc(const Params &p, const float *state, cudaStream_t st) {
+    RS_DISPATCH_NPASS(CC, p.R, return launch_load_t, (p, state, st));
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_load_checkpoint(const Params &p, const float *state, cudaStream_t st) {
+    RS_DISPATCH_CC(p.CC, return launch_load_cc, (p, state, st));
+    return cudaErrorInvalidValue;
+}
+
+// -------------------------------------------------------------------- init --
+// After the host zeroes the workspace: E4M3 scales start at 1 (an all-zero tile).
+__global__ void fill_kernel(float *x, size_t n, float v) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        x[i] = v;
+}
+
+cudaError_t launch_init(const Params &p, cudaStream_t st) {
+    if (p.copy_dtype == RS_E4M3) {
+        const size_t n = (size_t)p.B * p.H;
+        fill_kernel<<<(unsigned)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024), 256, 0, st>>>(p.scale, n, 1.f);
+        return cudaGetLastError();
+    }
+    return cudaSuccess;
+}
+
+}  // namespace rs

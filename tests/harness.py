@@ -1,0 +1,167 @@
+"""Helpers shared by the GPU parity tests: run a workload through the CUDA
+library and the same inputs through the fp64 oracle, then compare.
+
+Error metric (the pages fix none): the normwise relative error of every
+(sequence, head) output vector, ||y_gpu - y_oracle||_2 / ||y_oracle||_2 over its
+R elements; a test reports the maximum over vectors and steps.  The same ratio
+in the infinity norm (rel_err_inf) is reported as a diagnostic: with an fp8
+copy its worst row can exceed the E4M3 unit roundoff through cancellation in
+the row's dot product, which the 2-norm averages over the vector.
+"""
+import numpy as np
+import torch
+
+import oracle
+import rs_decode_outputs_b200 as rs
+from rs_decode_outputs_b200 import inputs as gen
+
+TOL_F32 = 1e-4    # fp32 checkpoint / outputs read the fp32 master
+TOL_BF16 = 2e-2   # bf16 output copy
+TOL_E4M3 = 6e-2   # fp8 E4M3 output copy with a per-(sequence, head) scale
+
+PARAM_SEED_OFFSET = 0
+STREAM_SEED_OFFSET = 10_000
+
+
+def f64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def rel_err(y, ref):
+    """max over leading dims of ||y - ref||_2 / ||ref||_2 along the last axis."""
+    y = np.asarray(y, np.float64)
+    ref = np.asarray(ref, np.float64)
+    num = np.sqrt(np.sum((y - ref) ** 2, axis=-1))
+    den = np.maximum(np.sqrt(np.sum(ref ** 2, axis=-1)), 1e-300)
+    return float(np.max(num / den))
+
+
+def rel_err_inf(y, ref):
+    """max over leading dims of ||y - ref||_inf / ||ref||_inf along the last axis."""
+    y = np.asarray(y, np.float64)
+    ref = np.asarray(ref, np.float64)
+    num = np.max(np.abs(y - ref), axis=-1)
+    den = np.maximum(np.max(np.abs(ref), axis=-1), 1e-300)
+    return float(np.max(num / den))
+
+
+def torch_dtype(code):
+    return {rs.RS_F32: torch.float32, rs.RS_BF16: torch.bfloat16}[code]
+
+
+# ------------------------------------------------------------------ Mamba-2
+
+class Mamba2Case:
+    """A Mamba-2 workload: params, an input stream, and oracle bookkeeping for a
+    set of sampled (sequence, head) pairs (all pairs when `pairs` is None)."""
+
+    def __init__(self, B, H, P, N, G, in_dtype, seed, device, pairs=None, gen_device=None):
+        self.B, self.H, self.P, self.N, self.G = B, H, P, N, G
+        self.device = torch.device(device)
+        gdev = torch.device(gen_device or "cpu")
+        self.A, self.D, dtb = gen.mamba2_params(H, seed + PARAM_SEED_OFFSET, gdev)
+        self.stream = gen.Mamba2Stream(B, H, P, N, G, torch_dtype(in_dtype), dtb,
+                                       seed + STREAM_SEED_OFFSET, gdev)
+        self.pairs = [(b, h) for b in range(B) for h in range(H)] if pairs is None else list(pairs)
+        self.pb = np.array([p[0] for p in self.pairs])
+        self.ph = np.array([p[1] for p in self.pairs])
+        self.pg = self.ph // (H // G)
+        self.hstate = np.zeros((len(self.pairs), P, N))
+
+    def draw(self, T):
+        s = self.stream.next(T)
+        return {k: v.to(self.device) for k, v in s.items()}
+
+    def pair_inputs(self, s):
+        """Oracle view of step dict s: per pair arrays [n, T, ...] in float64."""
+        x = f64(s["x"])[:, self.pb, self.ph, :].transpose(1, 0, 2)
+        dt = f64(s["dt"])[:, self.pb, self.ph].T
+        Bm = f64(s["B"])[:, self.pb, self.pg, :].transpose(1, 0, 2)
+        C = f64(s["C"])[:, self.pb, self.pg, :].transpose(1, 0, 2)
+        return x, dt, Bm, C
+
+    def oracle_run(self, s, advance=True, h=None):
+        """Eager fp64 outputs [T, n, P] for the pairs; advances the oracle state."""
+        x, dt, Bm, C = self.pair_inputs(s)
+        A = f64(self.A)[self.ph]
+        D = f64(self.D)[self.ph]
+        h0 = (self.hstate if h is None else h).copy()
+        y, h1 = oracle.mamba2_eager_batch(A, D, x, dt, Bm, C, h=h0)
+        if advance and h is None:
+            self.hstate = h1
+        return y.transpose(1, 0, 2), h1
+
+    def gpu_pairs(self, y):
+        """y [..., B, H, R] tensor -> [..., n, R] numpy (sampled pairs)."""
+        return f64(y)[..., self.pb, self.ph, :]
+
+
+# ---------------------------------------------------------------------- GDN
+
+class GdnCase:
+    def __init__(self, B, H, dk, dv, in_dtype, seed, device, pairs=None, gen_device=None,
+                 scale=1.0):
+        self.B, self.H, self.dk, self.dv = B, H, dk, dv
+        self.scale = scale
+        self.device = torch.device(device)
+        gdev = torch.device(gen_device or "cpu")
+        A_log, dtb = gen.gdn_params(H, seed + PARAM_SEED_OFFSET, gdev)
+        self.stream = gen.GdnStream(B, H, dk, dv, torch_dtype(in_dtype), A_log, dtb,
+                                    seed + STREAM_SEED_OFFSET, gdev)
+        self.pairs = [(b, h) for b in range(B) for h in range(H)] if pairs is None else list(pairs)
+        self.pb = np.array([p[0] for p in self.pairs])
+        self.ph = np.array([p[1] for p in self.pairs])
+        self.hstate = np.zeros((len(self.pairs), dv, dk))
+
+    def draw(self, T):
+        s = self.stream.next(T)
+        return {k: v.to(self.device) for k, v in s.items()}
+
+    def pair_inputs(self, s):
+        q = f64(s["q"])[:, self.pb, self.ph, :].transpose(1, 0, 2)
+        k = f64(s["k"])[:, self.pb, self.ph, :].transpose(1, 0, 2)
+        v = f64(s["v"])[:, self.pb, self.ph, :].transpose(1, 0, 2)
+        a = f64(s["alpha"])[:, self.pb, self.ph].T
+        b = f64(s["beta"])[:, self.pb, self.ph].T
+        return q, k, v, a, b
+
+    def oracle_run(self, s, advance=True, h=None):
+        q, k, v, a, b = self.pair_inputs(s)
+        h0 = (self.hstate if h is None else h).copy()
+        o, h1 = oracle.gdn_eager_batch(q, k, v, a, b, S=h0, scale=self.scale)
+        if advance and h is None:
+            self.hstate = h1
+        return o.transpose(1, 0, 2), h1
+
+    def gpu_pairs(self, y):
+        return f64(y)[..., self.pb, self.ph, :]
+
+
+# -------------------------------------------------------------- checks ----
+
+def check_copy_is_quantised_master(sess):
+    """No drift: the output copy is exactly the quantisation of the fp32 master
+    (bf16 RNE, or E4M3 with scale = absmax / 448 per tile)."""
+    cfg = sess.cfg
+    master = sess.master().detach().cpu().numpy().astype(np.float32)
+    if cfg.copy_dtype == rs.RS_BF16:
+        got = sess.copy().detach().cpu().view(torch.int16).numpy().view(np.uint16)
+        exp = oracle.bf16_rne(master)
+        assert np.array_equal(got, exp), f"{np.sum(got != exp)} bf16 codes differ"
+    elif cfg.copy_dtype == rs.RS_E4M3:
+        codes = sess.copy().detach().cpu().numpy()
+        scales = sess.scale().detach().cpu().numpy()
+        B, H = master.shape[:2]
+        for b in range(B):
+            for h in range(H):
+                c_exp, s_exp = oracle.e4m3_quantize_tile(master[b, h])
+                assert scales[b, h] == s_exp, (b, h, scales[b, h], s_exp)
+                assert np.array_equal(codes[b, h], c_exp), (b, h)
+
+
+def make_session(kind, B, H, R, CC, G=1, cap=16, npos_max=1, in_dtype=rs.RS_BF16,
+                 copy_dtype=rs.RS_BF16, out_dtype=rs.RS_F32, shared_lowp=0, A=None, D=None,
+                 gdn_scale=1.0, device="cuda"):
+    cfg = rs.make_config(kind, B, H, R, CC, G, cap, npos_max, in_dtype, copy_dtype, out_dtype,
+                         shared_lowp, gdn_scale)
+    return rs.ReplaySSM(cfg, A=A, D=D, device=device)

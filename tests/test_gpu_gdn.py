@@ -1,0 +1,131 @@
+"""GPU parity of the Gated DeltaNet path against the fp64 oracle (all calls go
+through the C interface of librs_b200.so)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rs_decode_outputs_b200 as rs
+from oracle.replay_model import RingPointers
+from tests.harness import (TOL_BF16, TOL_E4M3, TOL_F32, GdnCase, check_copy_is_quantised_master,
+                           make_session, rel_err)
+
+pytestmark = pytest.mark.gpu
+
+
+def decode_run(case, sess, steps, K, check_drift=False):
+    ptr = RingPointers(case.B, sess.cfg.cap)
+    worst = 0.0
+    for t in range(steps):
+        s = case.draw(1)
+        sess.append(s, 1)
+        ptr.append(1)
+        y = sess.decode()
+        ref, _ = case.oracle_run(s)
+        worst = max(worst, rel_err(case.gpu_pairs(y), ref[0]))
+        if ptr.length[0] >= K:
+            sess.commit(min_len=K)
+            ptr.commit(min_len=K)
+            if check_drift:
+                check_copy_is_quantised_master(sess)
+        head, tail = sess.read_ptrs()
+        assert np.array_equal(head, ptr.head) and np.array_equal(tail, ptr.tail), t
+    status, flags = sess.get_error()
+    assert status == rs.RS_OK and not flags.any()
+    return worst
+
+
+def test_tiny_gdn_fp32_from_zero(cuda_device):
+    """Test-only mirror of the Mamba-2 config 0: B=2, H=4, dk=dv=16, fp32, K=4, 32 steps."""
+    case = GdnCase(2, 4, 16, 16, rs.RS_F32, seed=100, device=cuda_device, scale=0.5)
+    sess = make_session(rs.RS_GDN, 2, 4, 16, 16, cap=4, in_dtype=rs.RS_F32,
+                        copy_dtype=rs.RS_NONE, gdn_scale=0.5)
+    err = decode_run(case, sess, 32, K=4)
+    assert err <= TOL_F32, err
+    m = sess.master().double().cpu().numpy()
+    assert rel_err(m.reshape(2, 4, -1), case.hstate.reshape(2, 4, -1)) <= 1e-5
+
+
+@pytest.mark.parametrize("copy,tol", [(rs.RS_BF16, TOL_BF16), (rs.RS_E4M3, TOL_E4M3),
+                                      (rs.RS_NONE, TOL_F32)])
+def test_ragged_shapes_with_copies(cuda_device, copy, tol):
+    B, H, dk, dv, K = 3, 5, 128, 72, 6
+    case = GdnCase(B, H, dk, dv, rs.RS_BF16, seed=111, device=cuda_device)
+    sess = make_session(rs.RS_GDN, B, H, dv, dk, cap=8, copy_dtype=copy)
+    state = torch.zeros(B, H, dv, dk, device=cuda_device)
+    pre = case.draw(30)
+    sess.eager_step(state, rs.RS_F32, pre, 30)
+    case.oracle_run(pre)
+    sess.load_checkpoint(state)
+    err = decode_run(case, sess, 25, K=K, check_drift=copy != rs.RS_NONE)
+    assert err <= tol, err
+
+
+def test_verify_rollback_spec_rounds(cuda_device):
+    B, H, dk, dv = 4, 3, 64, 64
+    case = GdnCase(B, H, dk, dv, rs.RS_BF16, seed=121, device=cuda_device)
+    sess = make_session(rs.RS_GDN, B, H, dv, dk, cap=16, npos_max=5, copy_dtype=rs.RS_BF16)
+    acc = rs.inputs.acceptance(12, B, 4, 0.7, seed=6)
+    ptr = RingPointers(B, 16)
+    worst = 0.0
+    for r in range(12):
+        s = case.draw(5)
+        sess.append(s, 5)
+        ptr.append(5)
+        y = sess.verify(5)
+        ref, _ = case.oracle_run(s, advance=False)
+        worst = max(worst, rel_err(case.gpu_pairs(y), ref))
+        a = acc[r].numpy()
+        sess.rollback(torch.tensor(4 - a, dtype=torch.int32, device=cuda_device))
+        ptr.rollback(4 - a)
+        q, k, v, al, be = case.pair_inputs(s)
+        for i, (b, h) in enumerate(case.pairs):
+            n = 1 + int(a[b])
+            _, case.hstate[i] = oracle.gdn_eager(q[i, :n], k[i, :n], v[i, :n], al[i, :n],
+                                                 be[i, :n], S0=case.hstate[i])
+        sess.commit(min_len=8)
+        ptr.commit(min_len=8)
+        head, tail = sess.read_ptrs()
+        assert np.array_equal(head, ptr.head) and np.array_equal(tail, ptr.tail), r
+    assert worst <= TOL_BF16, worst
+
+
+@pytest.mark.parametrize("sdt,tol", [(rs.RS_F32, TOL_F32), (rs.RS_BF16, 5e-2)])
+def test_eager_baseline_kernel(cuda_device, sdt, tol):
+    B, H, dk, dv = 3, 4, 128, 128
+    case = GdnCase(B, H, dk, dv, rs.RS_BF16, seed=151, device=cuda_device)
+    sess = make_session(rs.RS_GDN, B, H, dv, dk, cap=8)
+    state = torch.zeros(B, H, dv, dk, device=cuda_device,
+                        dtype=torch.float32 if sdt == rs.RS_F32 else torch.bfloat16)
+    worst = 0.0
+    for t in range(20):
+        s = case.draw(1)
+        y = sess.eager_step(state, sdt, s, 1)
+        ref, _ = case.oracle_run(s)
+        worst = max(worst, rel_err(case.gpu_pairs(y), ref))
+    s = case.draw(5)
+    y = sess.eager_step(state, sdt, s, 5)
+    ref, _ = case.oracle_run(s)
+    worst = max(worst, rel_err(case.gpu_pairs(y), ref))
+    assert worst <= tol, worst
+
+
+def test_shared_lowp_arm_runs_and_is_not_better(cuda_device):
+    """The comparison arm (one shared low-precision checkpoint that also serves
+    the updates) against the dual-precision arm, both E4M3, from the same
+    prefilled checkpoint: the dual arm stays within the fp8 tolerance and is
+    no worse than the shared arm."""
+    B, H, dk, dv, K = 2, 4, 64, 64, 4
+    errs = {}
+    for shared in (0, 1):
+        case = GdnCase(B, H, dk, dv, rs.RS_BF16, seed=161, device=cuda_device)
+        sess = make_session(rs.RS_GDN, B, H, dv, dk, cap=8, copy_dtype=rs.RS_E4M3,
+                            shared_lowp=shared)
+        state = torch.zeros(B, H, dv, dk, device=cuda_device)
+        pre = case.draw(64)
+        sess.eager_step(state, rs.RS_F32, pre, 64)
+        case.oracle_run(pre)
+        sess.load_checkpoint(state)
+        errs[shared] = decode_run(case, sess, 64, K=K)
+    assert errs[0] <= TOL_E4M3, errs
+    assert errs[0] <= errs[1] * 1.05, errs
