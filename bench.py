@@ -28,6 +28,9 @@ POOL = 256          # distinct decode steps of inputs kept resident (cycled)
 METRIC = "SSM-layer decode tokens/s at batch 256; achieved HBM GB/s vs B200 peak"
 UNIT = "tokens/s"
 WORKLOAD = "mamba2-decode-b256-h80-p64-n128-bf16copy-K8"
+# DRAM bytes (read + write) of one streaming-kernel launch on this workload,
+# from an ncu capture of the current kernel (None when not yet captured).
+TRAFFIC = None
 
 
 def parse():
@@ -36,6 +39,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=2048)
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", default="rs", choices=["rs", "reference"])
+    ap.add_argument("--prefill", type=int, default=PREFILL)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-work", type=float, default=20.0)
     return ap.parse_args()
@@ -192,13 +196,16 @@ def gpu_arm(args, rank, world):
                          copy_dtype=rs.RS_BF16, out_dtype=rs.RS_BF16)
     sess = rs.ReplaySSM(cfg, A=A, D=D, device=dev)
 
-    # prefill: 512 eager fp32 steps on a state tensor, then load it as the checkpoint
+    # prefill: eager fp32 steps on a state tensor, then load it as the checkpoint
     state = torch.zeros(B, H, P, N, device=dev)
     ypre = torch.empty(1, B, H, P, device=dev, dtype=torch.bfloat16)
-    for c in range(PREFILL // 64):
-        chunk = src.next(64)
-        for t in range(64):
+    left = args.prefill
+    while left > 0:
+        n = min(64, left)
+        chunk = src.next(n)
+        for t in range(n):
             sess.eager_step(state, rs.RS_F32, {k: v[t:t + 1] for k, v in chunk.items()}, 1, ypre)
+        left -= n
     sess.load_checkpoint(state)
     del state
 
@@ -207,19 +214,18 @@ def gpu_arm(args, rank, world):
     y = sess.new_out()
     h = sess.handle
 
+    ins = [rs.make_inputs(d) for d in steps_in]
+
     def step(i, ev=None):
-        rs.rs_append(h, rs.make_inputs(steps_in[i % POOL]), 1)
-        if ev is not None:
-            ev[0].record(stream)
-        rs.rs_decode_outputs(h, y)
-        if ev is not None:
-            ev[1].record(stream)
+        # one decode step: append this token's inputs and replay the outputs
+        # (prep kernel + streaming kernel), then commit every K_COMMIT steps
+        rs.rs_decode_step(h, ins[i % POOL], 1, y)
         if (i + 1) % K_COMMIT == 0:
             if ev is not None:
-                ev[2].record(stream)
+                ev[0].record(stream)
             rs.rs_commit(h, K_COMMIT)
             if ev is not None:
-                ev[3].record(stream)
+                ev[1].record(stream)
 
     i = 0
     for _ in range(args.warmup):
@@ -251,16 +257,23 @@ def gpu_arm(args, rank, world):
         ms = float(t.item())
         dist.barrier()
 
-    # pass 2: per-kernel durations (events around each launch) for the roofline
+    # pass 2: per-kernel durations for the roofline (the library's own events
+    # around its prep and streaming launches; events around each commit)
     nk = min(args.steps, 512)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nk)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(nk)]
     torch.cuda.synchronize()
+    rs.rs_profile_start(h, nk)
+    com_idx = []
     for j in range(nk):
+        if (i + 1) % K_COMMIT == 0:
+            com_idx.append(j)
         step(i, evs[j])
         i += 1
     torch.cuda.synchronize()
-    dec_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    com_ms = [e[2].elapsed_time(e[3]) for e, j in zip(evs, range(nk)) if (i - nk + j + 1) % K_COMMIT == 0]
+    ncalls, prep_total, stream_total = rs.rs_profile_stop(h)
+    prep_ms = prep_total / ncalls
+    stream_ms = stream_total / ncalls
+    com_ms = [evs[j][0].elapsed_time(evs[j][1]) for j in com_idx]
 
     # eager read-modify-write baseline on the same shape (fp32 state and bf16 state)
     eager = {}
@@ -287,6 +300,7 @@ def gpu_arm(args, rank, world):
     ne2e = min(args.steps, 256)
     host_in = [{k: v.cpu().pin_memory() for k, v in steps_in[j].items()} for j in range(min(POOL, ne2e))]
     dev_in = {k: torch.empty_like(v) for k, v in steps_in[0].items()}
+    dev_ins = rs.make_inputs(dev_in)
     y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host_in[0].values())
     d2h = y.numel() * y.element_size()
@@ -296,8 +310,7 @@ def gpu_arm(args, rank, world):
     for j in range(ne2e):
         for k, v in host_in[j % len(host_in)].items():
             dev_in[k].copy_(v, non_blocking=True)
-        rs.rs_append(h, rs.make_inputs(dev_in), 1)
-        rs.rs_decode_outputs(h, y)
+        rs.rs_decode_step(h, dev_ins, 1, y)
         if (i + 1) % K_COMMIT == 0:
             rs.rs_commit(h, K_COMMIT)
         i += 1
@@ -319,8 +332,7 @@ def gpu_arm(args, rank, world):
     hbm, peak_kind = peaks()
     copy_bytes = B * H * P * N * 2
     y_bytes = B * H * P * 2
-    dec_avg = statistics.mean(dec_ms)
-    achieved = (copy_bytes + y_bytes) / (dec_avg * 1e-3) / 1e9
+    achieved = (copy_bytes + y_bytes) / (stream_ms * 1e-3) / 1e9
     com_avg = statistics.mean(com_ms) if com_ms else float("nan")
     commit_bytes = B * H * P * N * (4 + 4 + 2)
     step_ms = ms / args.steps
@@ -332,15 +344,16 @@ def gpu_arm(args, rank, world):
         "data": "synthetic (seeded; Mamba-2 serving-shape distributions)",
         "config": {"workload": WORKLOAD, "global_batch": B * world, "batch_per_gpu": B,
                    "nheads": H, "headdim": P, "dstate": N, "ngroups": G, "commit_interval": K_COMMIT,
-                   "ring_cap": CAP, "prefill_tokens": PREFILL, "checkpoint": "fp32 master + bf16 copy",
+                   "ring_cap": CAP, "prefill_tokens": args.prefill, "checkpoint": "fp32 master + bf16 copy",
                    "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
                    "l2": "inputs larger than L2 (checkpoint copy 335 MB per step), no flush"},
-        "roofline": {"bound": "hbm", "kernel": "m2_outputs_kernel (output-only replay)",
+        "roofline": {"bound": "hbm", "kernel": "stream_outputs_kernel (output-only replay, Mamba-2)",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "traffic": None, "peak_source": peak_kind,
+                     "traffic": TRAFFIC, "peak_source": peak_kind,
                      "algorithmic_bytes_per_launch": copy_bytes + y_bytes,
-                     "avg_launch_us": dec_avg * 1e3},
-        "kernels": {"decode_us": dec_avg * 1e3, "commit_us": com_avg * 1e3,
+                     "avg_launch_us": stream_ms * 1e3},
+        "kernels": {"prep_us": prep_ms * 1e3, "stream_us": stream_ms * 1e3,
+                    "decode_us": (prep_ms + stream_ms) * 1e3, "commit_us": com_avg * 1e3,
                     "commit_gbs": commit_bytes / (com_avg * 1e-3) / 1e9 if com_ms else None,
                     "step_state_bytes_per_token": H * P * N * (2 + 10 / K_COMMIT),
                     "step_achieved_gbs": B * H * P * N * (2 + 10 / K_COMMIT) / (step_ms * 1e-3) / 1e9},

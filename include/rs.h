@@ -109,17 +109,27 @@ typedef struct {
 
 /* Byte offsets of the regions of a workspace (each 256-byte aligned; a region a
  * configuration does not use has size 0).  Tests and tools use this to view the
- * checkpoints and pointers; kernels get the same offsets. */
+ * checkpoints and pointers; kernels get the same offsets.
+ *
+ * The input ring keeps, per (sequence, head) or (sequence, group), one block of
+ * cap slots; the entry at logical position t sits in slot t mod cap.  Blocks
+ * are contiguous so that a whole block moves in one bulk copy; a block's stride
+ * is its size rounded up to 16 bytes.  capd = max(cap, 4). */
 typedef struct {
     size_t master, master_bytes;   /* fp32 [B][H][R][Cc]          (not with shared_lowp) */
     size_t copy, copy_bytes;       /* copy_dtype [B][H][R][Cc]    (not with RS_NONE)     */
     size_t scale, scale_bytes;     /* fp32 [B][H]                 (RS_E4M3 only)         */
-    size_t ring_a, ring_a_bytes;   /* Mamba-2 x [B][cap][H][P]   | GDN q [B][cap][H][dk] */
-    size_t ring_b, ring_b_bytes;   /* Mamba-2 dt [B][cap][H] f32 | GDN k [B][cap][H][dk] */
-    size_t ring_c, ring_c_bytes;   /* Mamba-2 B [B][cap][G][N]   | GDN v [B][cap][H][dv] */
-    size_t ring_d, ring_d_bytes;   /* Mamba-2 C [B][cap][G][N]   | GDN alpha [B][cap][H] */
-    size_t ring_e, ring_e_bytes;   /* (unused for Mamba-2)       | GDN beta [B][cap][H]  */
-    size_t head, tail, err, arrive;/* int32 / int32 / uint32 / uint32, each [B]          */
+    size_t ring_a, ring_a_bytes;   /* Mamba-2 x [B][H][cap][P]     | GDN q [B][H][cap][dk] */
+    size_t ring_b, ring_b_bytes;   /* Mamba-2 dt [B][H][capd] f32  | GDN k [B][H][cap][dk] */
+    size_t ring_c, ring_c_bytes;   /* Mamba-2 B [B][G][cap][N]     | GDN v [B][H][cap][dv] */
+    size_t ring_d, ring_d_bytes;   /* Mamba-2 C [B][G][cap][N]     | GDN alpha [B][H][capd] */
+    size_t ring_e, ring_e_bytes;   /* (unused for Mamba-2)         | GDN beta [B][H][capd]  */
+    size_t head, tail, err, arrive;/* int32 / int32 / uint32 / uint32, each [B]            */
+    size_t scratch, scratch_bytes; /* fp32 replay records, written and read inside one
+                                      output call (NP = npos_max rounded up to 1, 2, 5, 8):
+                                      Mamba-2: [B][G][NP Cc] group records, then
+                                      [B][H][8 + NP R] tile records; GDN: [B][H][8 + NP (R
+                                      + Cc)]; each record rounded up to 16 bytes          */
     size_t total;
 } rs_layout;
 
@@ -156,6 +166,16 @@ rs_status rs_append(rs_handle h, const rs_inputs *in, int T, rs_stream stream);
  * (the fp32 master when copy_dtype is RS_NONE).  y: out_dtype [B][H][R].
  * A sequence with an empty buffer gets zeros and RS_SEQ_ERR_EMPTY. */
 rs_status rs_decode_outputs(rs_handle h, void *y, rs_stream stream);
+
+/* One decode step in two kernels: append T >= 1 inputs per sequence (as
+ * rs_append) and compute the outputs at those T newest positions (as
+ * rs_verify_outputs with npos = T); T <= npos_max.  T = 1 is a plain decode
+ * step, y: out_dtype [B][H][R]; T > 1 verifies T speculative positions,
+ * y: [T][B][H][R].  The new inputs are read once, straight from `in`, and
+ * written into the ring by the same kernel that prepares the replay.  A
+ * sequence whose buffer would overflow is left unchanged, gets zeros and
+ * RS_SEQ_ERR_OVERFLOW. */
+rs_status rs_decode_step(rs_handle h, const rs_inputs *in, int T, void *y, rs_stream stream);
 
 /* Commit (How ReplaySSM works, step 3): for every sequence with
  * len >= max(min_len, 1) and, when mask is not NULL, mask[b] != 0 (int32 [B],
@@ -213,6 +233,17 @@ rs_status rs_read_ptrs(rs_handle h, int32_t *head_host, int32_t *tail_host, rs_s
 const char *rs_status_string(int status);
 const char *rs_last_cuda_error(void);     /* text of the last failing CUDA call */
 uint64_t rs_launch_count(void);           /* kernels launched by this library so far */
+
+/* Kernel timing of the output calls (rs_decode_outputs, rs_verify_outputs,
+ * rs_decode_step), which each run a small prep kernel and one streaming
+ * kernel.  rs_profile_start creates CUDA events for the next `max_calls`
+ * output calls of this handle (1..2^20; later calls are not timed);
+ * rs_profile_stop waits for them and returns the number of timed calls and
+ * the summed device time (ms) of the prep kernels and of the streaming
+ * kernels, then frees the events.  Either output pointer may be NULL.  Not
+ * thread-safe with concurrent calls on the same handle. */
+rs_status rs_profile_start(rs_handle h, int max_calls);
+rs_status rs_profile_stop(rs_handle h, int *calls, float *prep_ms, float *stream_ms);
 
 #ifdef __cplusplus
 }

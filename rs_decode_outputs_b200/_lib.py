@@ -51,7 +51,7 @@ _sz = ctypes.c_size_t
 _LAYOUT_FIELDS = ["master", "master_bytes", "copy", "copy_bytes", "scale", "scale_bytes",
                   "ring_a", "ring_a_bytes", "ring_b", "ring_b_bytes", "ring_c", "ring_c_bytes",
                   "ring_d", "ring_d_bytes", "ring_e", "ring_e_bytes", "head", "tail", "err",
-                  "arrive", "total"]
+                  "arrive", "scratch", "scratch_bytes", "total"]
 
 
 class RsLayout(ctypes.Structure):
@@ -61,7 +61,7 @@ class RsLayout(ctypes.Structure):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m rs_decode_outputs_b200.build` (nvcc, sm_100a)")
+                          "`python rs_decode_outputs_b200/build.py` (nvcc, sm_100a)")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i32, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_int
     P = ctypes.POINTER
@@ -73,6 +73,7 @@ def _load():
         "rs_load_checkpoint": [vp, vp, vp],
         "rs_append": [vp, P(RsInputs), i32, vp],
         "rs_decode_outputs": [vp, vp, vp],
+        "rs_decode_step": [vp, P(RsInputs), i32, vp, vp],
         "rs_commit": [vp, i32, vp, vp],
         "rs_verify_outputs": [vp, i32, vp, vp],
         "rs_rollback": [vp, vp, vp],
@@ -82,6 +83,8 @@ def _load():
         "rs_get_error": [vp, vp, vp, vp],
         "rs_clear_error": [vp, vp],
         "rs_read_ptrs": [vp, vp, vp, vp],
+        "rs_profile_start": [vp, i32],
+        "rs_profile_stop": [vp, vp, vp, vp],
     }
     for name, args in sigs.items():
         f = getattr(lib, name)
@@ -173,6 +176,12 @@ def rs_decode_outputs(h, y, stream=None):
     _check(_lib.rs_decode_outputs(h, _ptr(y), _stream(stream)), "rs_decode_outputs")
 
 
+def rs_decode_step(h, inputs, T, y, stream=None):
+    ins = inputs if isinstance(inputs, RsInputs) else make_inputs(inputs)
+    _check(_lib.rs_decode_step(h, ctypes.byref(ins), int(T), _ptr(y), _stream(stream)),
+           "rs_decode_step")
+
+
 def rs_commit(h, min_len=1, mask=None, stream=None):
     _check(_lib.rs_commit(h, int(min_len), _ptr(mask), _stream(stream)), "rs_commit")
 
@@ -225,3 +234,17 @@ def rs_read_ptrs(h, batch, stream=None):
 
 def rs_launch_count() -> int:
     return int(_lib.rs_launch_count())
+
+
+def rs_profile_start(h, max_calls):
+    _check(_lib.rs_profile_start(h, int(max_calls)), "rs_profile_start")
+
+
+def rs_profile_stop(h):
+    """Returns (timed calls, summed prep-kernel ms, summed streaming-kernel ms)."""
+    n = ctypes.c_int()
+    tp = ctypes.c_float()
+    ts = ctypes.c_float()
+    _check(_lib.rs_profile_stop(h, ctypes.byref(n), ctypes.byref(tp), ctypes.byref(ts)),
+           "rs_profile_stop")
+    return n.value, tp.value, ts.value

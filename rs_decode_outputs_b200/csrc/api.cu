@@ -8,6 +8,7 @@
 #include <vector>
 
 #include "launch.h"
+#include "outputs.cuh"
 #include "regtile.cuh"
 
 namespace {
@@ -83,24 +84,29 @@ rs_status make_layout(const rs_config *c, rs_layout *L) {
     put(L->master, L->master_bytes, c->shared_lowp ? 0 : 4 * E);
     put(L->copy, L->copy_bytes, c->copy_dtype == RS_NONE ? 0 : E * elem_bytes(c->copy_dtype));
     put(L->scale, L->scale_bytes, c->copy_dtype == RS_E4M3 ? 4 * B * H : 0);
+    const size_t capd = cap < 4 ? 4 : cap;
+    const size_t blk_r = (cap * R * ib + 15) / 16 * 16;   // x / v block per (b, h)
+    const size_t blk_c = cap * CC * ib;                   // q / k block per (b, h), B / C per (b, g)
     if (c->kind == RS_MAMBA2) {
-        put(L->ring_a, L->ring_a_bytes, B * cap * H * R * ib);
-        put(L->ring_b, L->ring_b_bytes, 4 * B * cap * H);
-        put(L->ring_c, L->ring_c_bytes, B * cap * G * CC * ib);
-        put(L->ring_d, L->ring_d_bytes, B * cap * G * CC * ib);
+        put(L->ring_a, L->ring_a_bytes, B * H * blk_r);
+        put(L->ring_b, L->ring_b_bytes, 4 * B * H * capd);
+        put(L->ring_c, L->ring_c_bytes, B * G * blk_c);
+        put(L->ring_d, L->ring_d_bytes, B * G * blk_c);
         put(L->ring_e, L->ring_e_bytes, 0);
     } else {
-        put(L->ring_a, L->ring_a_bytes, B * cap * H * CC * ib);
-        put(L->ring_b, L->ring_b_bytes, B * cap * H * CC * ib);
-        put(L->ring_c, L->ring_c_bytes, B * cap * H * R * ib);
-        put(L->ring_d, L->ring_d_bytes, 4 * B * cap * H);
-        put(L->ring_e, L->ring_e_bytes, 4 * B * cap * H);
+        put(L->ring_a, L->ring_a_bytes, B * H * blk_c);
+        put(L->ring_b, L->ring_b_bytes, B * H * blk_c);
+        put(L->ring_c, L->ring_c_bytes, B * H * blk_r);
+        put(L->ring_d, L->ring_d_bytes, 4 * B * H * capd);
+        put(L->ring_e, L->ring_e_bytes, 4 * B * H * capd);
     }
     size_t dummy;
     put(L->head, dummy, 4 * B);
     put(L->tail, dummy, 4 * B);
     put(L->err, dummy, 4 * B);
     put(L->arrive, dummy, 4 * B);
+    put(L->scratch, L->scratch_bytes,
+        4 * rs::scratch_floats(c->kind, c->batch, c->nheads, c->ngroups, c->npos_max, c->headdim, c->dstate));
     L->total = o;
     return RS_OK;
 }
@@ -118,7 +124,25 @@ struct rs_ctx {
     rs_layout lay;
     rs::Params p;
     int device;
+    // profiling: three events (before prep, between prep and stream, after stream) per output call
+    std::vector<cudaEvent_t> prof;
+    int prof_max = 0, prof_n = 0;
 };
+
+namespace {
+
+cudaEvent_t *prof_slot(rs_ctx *h) {
+    if (h->prof_n < h->prof_max) return &h->prof[3 * (h->prof_n++)];
+    return nullptr;
+}
+
+void prof_release(rs_ctx *h) {
+    for (cudaEvent_t e : h->prof) cudaEventDestroy(e);
+    h->prof.clear();
+    h->prof_max = h->prof_n = 0;
+}
+
+}  // namespace
 
 extern "C" {
 
@@ -163,6 +187,12 @@ rs_status rs_create(const rs_config *cfg, void *workspace, size_t workspace_byte
     p.heads_per_group = p.H / p.G;
     p.cap = cfg->cap;
     p.cap_mask = cfg->cap - 1;
+    p.capd = cfg->cap < 4 ? 4 : cfg->cap;
+    {
+        const int ib = elem_bytes(cfg->in_dtype);
+        p.blk_r = ((size_t)cfg->cap * cfg->headdim * ib + 15) / 16 * 16;
+        p.blk_c = (size_t)cfg->cap * cfg->dstate * ib;
+    }
     p.in_dtype = cfg->in_dtype;
     p.out_dtype = cfg->out_dtype;
     p.copy_dtype = cfg->copy_dtype;
@@ -182,15 +212,23 @@ rs_status rs_create(const rs_config *cfg, void *workspace, size_t workspace_byte
     p.arrive = reinterpret_cast<uint32_t *>(ws + L.arrive);
     p.A = A;
     p.D = D;
+    p.rec = reinterpret_cast<float *>(ws + L.scratch);
+    p.rec_tile_off = cfg->kind == RS_MAMBA2
+                         ? (size_t)p.B * p.G * rs::group_rec_floats(rs::prep_np(cfg->npos_max), p.CC)
+                         : 0;
 
     cudaError_t e = cudaGetDevice(&h->device);
     if (e != cudaSuccess) { delete h; return cuda_fail(e, "cudaGetDevice"); }
     int optin = 0;
     e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device);
     if (e != cudaSuccess) { delete h; return cuda_fail(e, "cudaDeviceGetAttribute"); }
-    const size_t need_out = cfg->kind == RS_MAMBA2 ? rs::m2_outputs_smem(p, 8) : rs::gdn_outputs_smem(p, 8);
-    const size_t need_commit = cfg->kind == RS_MAMBA2 ? rs::m2_commit_smem(p) : rs::gdn_commit_smem(p);
-    if (need_out > (size_t)optin - 1024 || need_commit > (size_t)optin - 1024) {
+    size_t need = cfg->kind == RS_MAMBA2 ? rs::m2_commit_smem(p) : rs::gdn_commit_smem(p);
+    for (int np = 1; np <= cfg->npos_max; ++np) {   // every output-position count a call may use
+        const size_t a = rs::stream_outputs_smem(p, np), b = rs::prep_smem(p, rs::prep_np(np));
+        need = a > need ? a : need;
+        need = b > need ? b : need;
+    }
+    if (need > (size_t)optin) {
         delete h;
         return RS_ERR_UNSUPPORTED;
     }
@@ -206,7 +244,48 @@ rs_status rs_create(const rs_config *cfg, void *workspace, size_t workspace_byte
 }
 
 rs_status rs_destroy(rs_handle h) {
+    if (h) prof_release(h);
     delete h;
+    return RS_OK;
+}
+
+rs_status rs_profile_start(rs_handle h, int max_calls) {
+    if (!h || max_calls < 1 || max_calls > (1 << 20)) return RS_ERR_ARG;
+    prof_release(h);
+    h->prof.resize(3 * (size_t)max_calls);
+    for (size_t i = 0; i < h->prof.size(); ++i) {
+        cudaError_t e = cudaEventCreate(&h->prof[i]);
+        if (e != cudaSuccess) {
+            h->prof.resize(i);
+            prof_release(h);
+            return cuda_fail(e, "cudaEventCreate");
+        }
+    }
+    h->prof_max = max_calls;
+    h->prof_n = 0;
+    return RS_OK;
+}
+
+rs_status rs_profile_stop(rs_handle h, int *calls, float *prep_ms, float *stream_ms) {
+    if (!h) return RS_ERR_ARG;
+    float tp = 0.f, ts = 0.f;
+    for (int c = 0; c < h->prof_n; ++c) {
+        cudaEvent_t *ev = &h->prof[3 * (size_t)c];
+        cudaError_t e = cudaEventSynchronize(ev[2]);
+        float a = 0.f, b = 0.f;
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&a, ev[0], ev[1]);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&b, ev[1], ev[2]);
+        if (e != cudaSuccess) {
+            prof_release(h);
+            return cuda_fail(e, "profile events");
+        }
+        tp += a;
+        ts += b;
+    }
+    if (calls) *calls = h->prof_n;
+    if (prep_ms) *prep_ms = tp;
+    if (stream_ms) *stream_ms = ts;
+    prof_release(h);
     return RS_OK;
 }
 
@@ -225,13 +304,21 @@ rs_status rs_append(rs_handle h, const rs_inputs *in, int T, rs_stream stream) {
 
 static rs_status outputs(rs_handle h, int npos, void *y, rs_stream stream) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (h->cfg.kind == RS_MAMBA2) return launched(rs::launch_m2_outputs(h->p, npos, y, st), "m2_outputs");
-    return launched(rs::launch_gdn_outputs(h->p, npos, y, st), "gdn_outputs");
+    const rs_inputs none{};
+    return launched(rs::launch_outputs(h->p, npos, 0, none, y, st, prof_slot(h)), "outputs", 2);
 }
 
 rs_status rs_decode_outputs(rs_handle h, void *y, rs_stream stream) {
     if (!h || !y) return RS_ERR_ARG;
     return outputs(h, 1, y, stream);
+}
+
+rs_status rs_decode_step(rs_handle h, const rs_inputs *in, int T, void *y, rs_stream stream) {
+    if (!h || !y || !has_inputs(h->cfg.kind, in)) return RS_ERR_ARG;
+    if (T < 1) return RS_ERR_ARG;
+    if (T > h->cfg.npos_max || T > h->cfg.cap) return RS_ERR_CAPACITY;
+    return launched(rs::launch_outputs(h->p, T, T, *in, y, static_cast<cudaStream_t>(stream), prof_slot(h)),
+                    "decode_step", 2);
 }
 
 rs_status rs_verify_outputs(rs_handle h, int npos, void *y, rs_stream stream) {

@@ -16,9 +16,10 @@ namespace rs {
 // Everything a kernel needs to find a handle's data.  Built on the host from the
 // workspace layout; passed by value.
 struct Params {
-    int kind, B, H, R, CC, G, cap, cap_mask, heads_per_group;
+    int kind, B, H, R, CC, G, cap, cap_mask, heads_per_group, capd;
     int in_dtype, out_dtype, copy_dtype, shared_lowp;
     float gdn_scale;
+    size_t blk_r, blk_c;   // ring block strides in bytes: R-wide rows (x, v), CC-wide rows (q, k, B, C)
     float *master;       // fp32 [B][H][R][CC] (NULL with shared_lowp)
     void *copy;          // copy_dtype [B][H][R][CC] (NULL with RS_NONE)
     float *scale;        // fp32 [B][H] (E4M3)
@@ -26,6 +27,8 @@ struct Params {
     int32_t *head, *tail;
     uint32_t *err, *arrive;
     const float *A, *D;  // Mamba-2 [H]
+    float *rec;          // scratch: Mamba-2 group records, then one replay record per (b, h) tile
+    size_t rec_tile_off; // floats from rec to the first tile record
 };
 
 // Threads of the CTAs that hold a state tile in registers.
@@ -45,6 +48,15 @@ __device__ __forceinline__ void st_out(void *p, size_t i, float v, int dtype) {
     if (dtype == RS_BF16) static_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(v);
     else static_cast<float *>(p)[i] = v;
 }
+
+// Element `i` of a shared-memory array of the input dtype, as float.
+__device__ __forceinline__ float lds_in(const void *smem_ptr, size_t i, int dtype) {
+    if (dtype == RS_BF16)
+        return __uint_as_float(static_cast<uint32_t>(static_cast<const unsigned short *>(smem_ptr)[i]) << 16);
+    return static_cast<const float *>(smem_ptr)[i];
+}
+
+__device__ __forceinline__ float lds_f32(const float *smem_ptr, size_t i) { return smem_ptr[i]; }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -109,6 +121,18 @@ struct Geom {
     static_assert(CHUNKS % TPR == 0, "chunks must split evenly");
 };
 
+// Two fp32 fused multiply-adds in one packed instruction: a * b + c elementwise.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    unsigned long long x, y, z, r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(y) : "f"(b.x), "f"(b.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(z) : "f"(c.x), "f"(c.y));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(x), "l"(y), "l"(z));
+    float2 o;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(o.x), "=f"(o.y) : "l"(r));
+    return o;
+}
+
 // Sum over the TPR lanes that share a row (TPR a power of two <= 8, aligned).
 template <int TPR>
 __device__ __forceinline__ float row_sum(float v) {
@@ -149,14 +173,17 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
                  : "memory");
 }
 
+// One bounded test of a barrier phase.  The thread may sleep in the hardware
+// for up to the hinted time (nanoseconds) while the phase is incomplete, so a
+// waiting warp does not keep re-issuing the test.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
         : "memory");
     return ok != 0;
 }
@@ -181,6 +208,20 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src, uint32
         " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst_smem)),
         "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
+}
+
+// Asynchronous 16-byte global -> shared copy through the L1 path (both
+// addresses 16-byte aligned); completion by cp_async_wait_all.
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *smem_dst, const void *gsrc) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
 // L2 policy for data streamed once per step (the checkpoints): evict first, so

@@ -20,191 +20,6 @@
 
 namespace rs {
 
-struct GdnOutSmem {
-    size_t alpha, beta, q, coef, mul, z, kraw, vraw, total;
-};
-
-__host__ __device__ inline GdnOutSmem gdn_out_smem(size_t tile_bytes, int cap, int CC, int R,
-                                                   int NP, int in_bytes) {
-    GdnOutSmem s;
-    size_t o = align_up(tile_bytes, 128);
-    s.alpha = o; o = align_up(o + 4 * (size_t)cap, 16);
-    s.beta = o;  o = align_up(o + 4 * (size_t)cap, 16);
-    s.q = o;     o = align_up(o + 4 * (size_t)NP * CC, 16);
-    s.coef = o;  o = align_up(o + 4 * (size_t)NP * cap, 16);
-    s.mul = o;   o = align_up(o + 4 * (size_t)NP, 16);
-    s.z = o;     o = align_up(o + 4 * (size_t)NP * R, 16);
-    s.kraw = o;  o = align_up(o + (size_t)in_bytes * cap * CC, 16);
-    s.vraw = o;  o = align_up(o + (size_t)in_bytes * cap * R, 16);
-    s.total = o;
-    return s;
-}
-
-// ------------------------------------------------------------- outputs ----
-
-template <int CC, typename TS, int NP>
-__global__ void __launch_bounds__(kOutThreads)
-gdn_outputs_kernel(const Params p, const void *__restrict__ state, int npos, void *y) {
-    extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ uint64_t bar;
-
-    const int R = p.R, H = p.H, cap = p.cap;
-    const int tile = blockIdx.x;
-    const int b = tile / H, h = tile % H;
-    const int in_bytes = p.in_dtype == RS_BF16 ? 2 : 4;
-    const uint32_t tile_bytes = static_cast<uint32_t>(R) * CC * TS::bytes;
-    const GdnOutSmem L_ = gdn_out_smem(tile_bytes, cap, CC, R, NP, in_bytes);
-    float *s_alpha = reinterpret_cast<float *>(smem + L_.alpha);
-    float *s_beta = reinterpret_cast<float *>(smem + L_.beta);
-    float *s_q = reinterpret_cast<float *>(smem + L_.q);
-    float *s_coef = reinterpret_cast<float *>(smem + L_.coef);
-    float *s_mul = reinterpret_cast<float *>(smem + L_.mul);
-    float *s_z = reinterpret_cast<float *>(smem + L_.z);
-    unsigned char *s_k = smem + L_.kraw;
-    unsigned char *s_v = smem + L_.vraw;
-
-    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-    constexpr int nwarps = kOutThreads / 32;
-
-    if (tid == 0) {
-        mbar_init(&bar, 1);
-        bulk_tile_g2s(smem, static_cast<const unsigned char *>(state) + (size_t)tile * tile_bytes,
-                      tile_bytes, &bar, policy_evict_first());
-    }
-
-    const int head = p.head[b];
-    const int L = p.tail[b] - head;
-    const bool ok = npos >= 1 && L >= npos && L <= cap;
-    const size_t ring_bh = (size_t)b * cap;
-
-    if (ok) {
-        for (int i = tid; i < L; i += kOutThreads) {
-            const size_t at = (ring_bh + ((head + i) & p.cap_mask)) * H + h;
-            s_alpha[i] = static_cast<const float *>(p.rd)[at];
-            s_beta[i] = static_cast<const float *>(p.re)[at];
-        }
-        const int kchunks = CC * in_bytes / 16;
-        for (int q = tid; q < L * kchunks; q += kOutThreads) {
-            const int i = q / kchunks, w = q % kchunks;
-            const size_t at = ((ring_bh + ((head + i) & p.cap_mask)) * H + h) * CC;
-            reinterpret_cast<uint4 *>(s_k + (size_t)i * CC * in_bytes)[w] =
-                reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(p.rb) + at * in_bytes)[w];
-        }
-        for (int q = tid; q < L * R; q += kOutThreads) {
-            const int i = q / R, r = q % R;
-            const size_t src = ((ring_bh + ((head + i) & p.cap_mask)) * H + h) * R + r;
-            if (in_bytes == 2)
-                reinterpret_cast<uint16_t *>(s_v)[q] = static_cast<const uint16_t *>(p.rc)[src];
-            else
-                reinterpret_cast<float *>(s_v)[q] = static_cast<const float *>(p.rc)[src];
-        }
-        for (int q = tid; q < npos * CC; q += kOutThreads) {
-            const int j = q / CC, c = q % CC;
-            const int slot = (head + L - npos + j) & p.cap_mask;
-            s_q[q] = ld_in(p.ra, ((ring_bh + slot) * H + h) * CC + c, p.in_dtype);
-        }
-    }
-    __syncthreads();
-
-    if (ok) {
-        // Backward sweep for each output position (one warp per position).
-        constexpr int UPL = (CC + 31) / 32;
-        for (int j = warp; j < npos; j += nwarps) {
-            const int e = L - npos + j;
-            float u[UPL];
-#pragma unroll
-            for (int m = 0; m < UPL; ++m) {
-                const int c = lane + 32 * m;
-                u[m] = c < CC ? s_q[j * CC + c] : 0.f;
-            }
-            for (int i = e; i >= 0; --i) {
-                float kr[UPL];
-                float ku = 0.f;
-#pragma unroll
-                for (int m = 0; m < UPL; ++m) {
-                    const int c = lane + 32 * m;
-                    kr[m] = c < CC ? ld_in(s_k, (size_t)i * CC + c, p.in_dtype) : 0.f;
-                    ku = fmaf(kr[m], u[m], ku);
-                }
-                ku = warp_sum(ku);
-                const float a = s_alpha[i], f = s_beta[i] * ku;
-                if (lane == 0) s_coef[j * cap + i] = f;
-#pragma unroll
-                for (int m = 0; m < UPL; ++m) u[m] = a * fmaf(-f, kr[m], u[m]);
-            }
-            __syncwarp();
-#pragma unroll
-            for (int m = 0; m < UPL; ++m) {
-                const int c = lane + 32 * m;
-                if (c < CC) s_q[j * CC + c] = u[m];
-            }
-        }
-        const float sc = p.gdn_scale;
-        if (tid < npos) s_mul[tid] = sc * (p.copy_dtype == RS_E4M3 ? p.scale[tile] : 1.f);
-    }
-    __syncthreads();
-
-    if (ok) {
-        const float sc = p.gdn_scale;
-        for (int q = tid; q < npos * R; q += kOutThreads) {
-            const int j = q / R, r = q % R, e = L - npos + j;
-            float acc = 0.f;
-            for (int i = 0; i <= e; ++i) acc = fmaf(s_coef[j * cap + i], ld_in(s_v, (size_t)i * R + r, p.in_dtype), acc);
-            s_z[q] = sc * acc;
-        }
-    }
-
-    const bool arrived = mbar_wait_bounded(&bar, 0);
-    __syncthreads();
-    const size_t y_pos_stride = (size_t)p.B * H * R;
-    const size_t y_off = (size_t)tile * R;
-    if (!ok || !arrived) {
-        zero_outputs(R, npos, y, y_pos_stride, y_off, p.out_dtype);
-        if (tid == 0) atomicOr(&p.err[b], !arrived ? RS_SEQ_ERR_TIMEOUT : RS_SEQ_ERR_EMPTY);
-        return;
-    }
-    tile_matvec<CC, TS, NP>(smem, R, s_q, npos, s_mul, s_z, y, y_pos_stride, y_off, p.out_dtype);
-}
-
-size_t gdn_outputs_smem(const Params &p, int NP) {
-    const int eb = p.copy_dtype == RS_BF16 ? 2 : p.copy_dtype == RS_E4M3 ? 1 : 4;
-    return gdn_out_smem((size_t)p.R * p.CC * eb, p.cap, p.CC, p.R, NP,
-                        p.in_dtype == RS_BF16 ? 2 : 4).total;
-}
-
-template <int CC, typename TS, int NP>
-static cudaError_t launch_gdn_out_t(const Params &p, int npos, void *y, cudaStream_t st) {
-    const void *state = p.copy_dtype == RS_NONE ? static_cast<const void *>(p.master) : p.copy;
-    const size_t smem = gdn_outputs_smem(p, NP);
-    auto k = gdn_outputs_kernel<CC, TS, NP>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k<<<p.B * p.H, kOutThreads, smem, st>>>(p, state, npos, y);
-    return cudaGetLastError();
-}
-
-template <int CC, typename TS>
-static cudaError_t launch_gdn_out_np(const Params &p, int npos, void *y, cudaStream_t st) {
-    if (npos <= 1) return launch_gdn_out_t<CC, TS, 1>(p, npos, y, st);
-    if (npos <= 2) return launch_gdn_out_t<CC, TS, 2>(p, npos, y, st);
-    if (npos <= 4) return launch_gdn_out_t<CC, TS, 4>(p, npos, y, st);
-    return launch_gdn_out_t<CC, TS, 8>(p, npos, y, st);
-}
-
-template <int CC>
-static cudaError_t launch_gdn_out_cc(const Params &p, int npos, void *y, cudaStream_t st) {
-    switch (p.copy_dtype) {
-        case RS_BF16: return launch_gdn_out_np<CC, StBF16>(p, npos, y, st);
-        case RS_E4M3: return launch_gdn_out_np<CC, StE4M3>(p, npos, y, st);
-        default: return launch_gdn_out_np<CC, StF32>(p, npos, y, st);
-    }
-}
-
-cudaError_t launch_gdn_outputs(const Params &p, int npos, void *y, cudaStream_t st) {
-    RS_DISPATCH_CC(p.CC, return launch_gdn_out_cc, (p, npos, y, st));
-    return cudaErrorInvalidValue;
-}
-
 // -------------------------------------------------------------- commit ----
 // Fold the buffer into the fp32 master row by row, in buffer order, with the
 // tile in registers; rewrite master and copy; the last CTA of a sequence moves
@@ -228,8 +43,13 @@ gdn_commit_kernel(const Params p, int min_len, const int32_t *__restrict__ mask)
     float *s_beta = s_alpha + cap;
     float *s_v = s_beta + cap;  // [cap][R]
     unsigned char *s_k = smem + align_up(4 * (2 * (size_t)cap + (size_t)cap * R), 16);  // [cap][CC]
-    const size_t ring_bh = (size_t)b * cap;
     const int tid = threadIdx.x;
+    // this head's ring blocks
+    const size_t bh = (size_t)b * H + h;
+    const unsigned char *kblk = static_cast<const unsigned char *>(p.rb) + bh * p.blk_c;
+    const unsigned char *vblk = static_cast<const unsigned char *>(p.rc) + bh * p.blk_r;
+    const float *ablk = static_cast<const float *>(p.rd) + bh * p.capd;
+    const float *bblk = static_cast<const float *>(p.re) + bh * p.capd;
 
     T t;
     t.init(R);
@@ -237,20 +57,19 @@ gdn_commit_kernel(const Params p, int min_len, const int32_t *__restrict__ mask)
     else t.load_f32(p.master + (size_t)tile * R * CC);
 
     for (int i = tid; i < L; i += kTileThreads) {
-        const size_t at = (ring_bh + ((head + i) & p.cap_mask)) * H + h;
-        s_alpha[i] = static_cast<const float *>(p.rd)[at];
-        s_beta[i] = static_cast<const float *>(p.re)[at];
+        const int slot = (head + i) & p.cap_mask;
+        s_alpha[i] = ablk[slot];
+        s_beta[i] = bblk[slot];
     }
-    const int kchunks = CC * in_bytes / 16;
-    for (int q = tid; q < L * kchunks; q += kTileThreads) {
-        const int i = q / kchunks, w = q % kchunks;
-        const size_t at = ((ring_bh + ((head + i) & p.cap_mask)) * H + h) * CC;
-        reinterpret_cast<uint4 *>(s_k + (size_t)i * CC * in_bytes)[w] =
-            reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(p.rb) + at * in_bytes)[w];
+    const int kshift = __ffs(CC * in_bytes / 16) - 1;   // 16-byte pieces per row, log2
+    for (int q = tid; q < (L << kshift); q += kTileThreads) {
+        const int i = q >> kshift, w = q & ((1 << kshift) - 1);
+        const unsigned char *src = kblk + (size_t)((head + i) & p.cap_mask) * CC * in_bytes;
+        reinterpret_cast<uint4 *>(s_k + (size_t)i * CC * in_bytes)[w] = reinterpret_cast<const uint4 *>(src)[w];
     }
-    for (int q = tid; q < L * R; q += kTileThreads) {
-        const int i = q / R, r = q % R;
-        s_v[q] = ld_in(p.rc, ((ring_bh + ((head + i) & p.cap_mask)) * H + h) * R + r, p.in_dtype);
+    for (int i = tid >> 5; i < L; i += kTileThreads / 32) {
+        const unsigned char *row = vblk + (size_t)((head + i) & p.cap_mask) * R * in_bytes;
+        for (int r = tid & 31; r < R; r += 32) s_v[i * R + r] = ld_in(row, r, p.in_dtype);
     }
     __syncthreads();
 

@@ -5,15 +5,17 @@
 
 #include "common.cuh"
 
-// Instantiate a launcher for each supported tile width (columns of a state tile).
-#define RS_DISPATCH_CC(cc, RET_FN, ARGS) \
-    switch (cc) {                        \
-        case 16: RET_FN<16> ARGS;        \
-        case 32: RET_FN<32> ARGS;        \
-        case 64: RET_FN<64> ARGS;        \
-        case 128: RET_FN<128> ARGS;      \
-        case 256: RET_FN<256> ARGS;      \
-        default: break;                  \
+// Instantiate a launcher for each supported tile width (columns of a state
+// tile).  RET_FN is either `return f` or an assignment `e = f`; each case ends
+// with a break, so exactly one instantiation runs.
+#define RS_DISPATCH_CC(cc, RET_FN, ARGS)        \
+    switch (cc) {                               \
+        case 16: { RET_FN<16> ARGS; } break;    \
+        case 32: { RET_FN<32> ARGS; } break;    \
+        case 64: { RET_FN<64> ARGS; } break;    \
+        case 128: { RET_FN<128> ARGS; } break;  \
+        case 256: { RET_FN<256> ARGS; } break;  \
+        default: break;                         \
     }
 
 // Rows of a register-resident tile each thread holds: ceil(R / rows-per-pass),
@@ -35,20 +37,27 @@
 
 namespace rs {
 
+// Output-only replay / verification (both kinds): the prep kernel writes one
+// record per tile into p.rec, then the streaming pass reads every checkpoint
+// tile once.  launch_outputs does both.
+cudaError_t launch_prep(const Params &p, int npos, int T, const rs_inputs &in, cudaStream_t st);
+// ev (may be NULL): three events recorded before the prep kernel, between the
+// two kernels and after the streaming kernel.
+cudaError_t launch_outputs(const Params &p, int npos, int T, const rs_inputs &in, void *y, cudaStream_t st,
+                           cudaEvent_t *ev = nullptr);
+size_t prep_smem(const Params &p, int NP);
+size_t stream_outputs_smem(const Params &p, int npos);
+
 // Mamba-2
-cudaError_t launch_m2_outputs(const Params &p, int npos, void *y, cudaStream_t st);
 cudaError_t launch_m2_commit(const Params &p, int min_len, const int32_t *mask, cudaStream_t st);
 cudaError_t launch_m2_eager(const Params &p, void *state, int sdt, const rs_inputs &in, int T,
                             void *y, const int32_t *cur, int nslots, cudaStream_t st);
-size_t m2_outputs_smem(const Params &p, int NP);
 size_t m2_commit_smem(const Params &p);
 
 // Gated DeltaNet
-cudaError_t launch_gdn_outputs(const Params &p, int npos, void *y, cudaStream_t st);
 cudaError_t launch_gdn_commit(const Params &p, int min_len, const int32_t *mask, cudaStream_t st);
 cudaError_t launch_gdn_eager(const Params &p, void *state, int sdt, const rs_inputs &in, int T,
                              void *y, const int32_t *cur, int nslots, cudaStream_t st);
-size_t gdn_outputs_smem(const Params &p, int NP);
 size_t gdn_commit_smem(const Params &p);
 
 // Ring / pointers / checkpoints (both kinds)

@@ -22,6 +22,22 @@ __device__ __forceinline__ void copy_coop(void *dst, const void *src, size_t nby
     }
 }
 
+// Copy one row of nbytes (a multiple of 2) with the 32 lanes of a warp, in the
+// widest pieces both ends allow.
+__device__ __forceinline__ void warp_copy(void *dst, const void *src, size_t nbytes, int lane) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src) | nbytes;
+    if ((a & 15) == 0) {
+        for (size_t i = lane; i < nbytes / 16; i += 32)
+            static_cast<uint4 *>(dst)[i] = static_cast<const uint4 *>(src)[i];
+    } else if ((a & 3) == 0) {
+        for (size_t i = lane; i < nbytes / 4; i += 32)
+            static_cast<uint32_t *>(dst)[i] = static_cast<const uint32_t *>(src)[i];
+    } else {
+        for (size_t i = lane; i < nbytes / 2; i += 32)
+            static_cast<uint16_t *>(dst)[i] = static_cast<const uint16_t *>(src)[i];
+    }
+}
+
 // ----------------------------------------------------------------- append --
 // One CTA per sequence ("ReplaySSM for hybrid SSM-Transformer stacks", How
 // ReplaySSM works, step 2: append the step's SSM input to the buffer).  Writes
@@ -36,22 +52,43 @@ __global__ void __launch_bounds__(256) append_kernel(const Params p, rs_inputs i
     }
     const int H = p.H, R = p.R, CC = p.CC, Bn = p.B;
     const size_t ib = p.in_dtype == RS_BF16 ? 2 : 4;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const size_t rrow = (size_t)R * ib, crow = (size_t)CC * ib;   // bytes of one ring row
     for (int t = 0; t < T; ++t) {
-        const size_t row = (size_t)b * p.cap + ((tail + t) & p.cap_mask);   // ring row of this entry
-        const size_t src = (size_t)t * Bn + b;                              // input row [t][b]
-        if (kind == RS_MAMBA2) {
-            const size_t nx = (size_t)H * R, nbc = (size_t)p.G * CC;
-            copy_coop(static_cast<char *>(p.ra) + row * nx * ib, static_cast<const char *>(in.x) + src * nx * ib, nx * ib);
-            copy_coop(static_cast<float *>(p.rb) + row * H, in.dt + src * H, (size_t)H * 4);
-            copy_coop(static_cast<char *>(p.rc) + row * nbc * ib, static_cast<const char *>(in.B) + src * nbc * ib, nbc * ib);
-            copy_coop(static_cast<char *>(p.rd) + row * nbc * ib, static_cast<const char *>(in.C) + src * nbc * ib, nbc * ib);
-        } else {
-            const size_t nk = (size_t)H * CC, nv = (size_t)H * R;
-            copy_coop(static_cast<char *>(p.ra) + row * nk * ib, static_cast<const char *>(in.q) + src * nk * ib, nk * ib);
-            copy_coop(static_cast<char *>(p.rb) + row * nk * ib, static_cast<const char *>(in.k) + src * nk * ib, nk * ib);
-            copy_coop(static_cast<char *>(p.rc) + row * nv * ib, static_cast<const char *>(in.v) + src * nv * ib, nv * ib);
-            copy_coop(static_cast<float *>(p.rd) + row * H, in.alpha + src * H, (size_t)H * 4);
-            copy_coop(static_cast<float *>(p.re) + row * H, in.beta + src * H, (size_t)H * 4);
+        const int slot = (tail + t) & p.cap_mask;
+        const size_t src = (size_t)t * Bn + b;   // input row [t][b]
+        // per-head rows (one warp per row) and per-head scalars
+        for (int h = warp; h < H; h += nw) {
+            const size_t bh = (size_t)b * H + h;
+            if (kind == RS_MAMBA2) {
+                warp_copy(static_cast<char *>(p.ra) + bh * p.blk_r + slot * rrow,
+                          static_cast<const char *>(in.x) + (src * H + h) * rrow, rrow, lane);
+            } else {
+                warp_copy(static_cast<char *>(p.ra) + bh * p.blk_c + slot * crow,
+                          static_cast<const char *>(in.q) + (src * H + h) * crow, crow, lane);
+                warp_copy(static_cast<char *>(p.rb) + bh * p.blk_c + slot * crow,
+                          static_cast<const char *>(in.k) + (src * H + h) * crow, crow, lane);
+                warp_copy(static_cast<char *>(p.rc) + bh * p.blk_r + slot * rrow,
+                          static_cast<const char *>(in.v) + (src * H + h) * rrow, rrow, lane);
+            }
+        }
+        for (int h = threadIdx.x; h < H; h += blockDim.x) {
+            const size_t at = ((size_t)b * H + h) * p.capd + slot;
+            if (kind == RS_MAMBA2) {
+                static_cast<float *>(p.rb)[at] = in.dt[src * H + h];
+            } else {
+                static_cast<float *>(p.rd)[at] = in.alpha[src * H + h];
+                static_cast<float *>(p.re)[at] = in.beta[src * H + h];
+            }
+        }
+        if (kind == RS_MAMBA2) {   // per-group rows of B and C
+            for (int g = warp; g < p.G; g += nw) {
+                const size_t bg = (size_t)b * p.G + g;
+                warp_copy(static_cast<char *>(p.rc) + bg * p.blk_c + slot * crow,
+                          static_cast<const char *>(in.B) + (src * p.G + g) * crow, crow, lane);
+                warp_copy(static_cast<char *>(p.rd) + bg * p.blk_c + slot * crow,
+                          static_cast<const char *>(in.C) + (src * p.G + g) * crow, crow, lane);
+            }
         }
     }
     __syncthreads();

@@ -1,0 +1,323 @@
+// The streaming half of the output-only kernels (decode and multi-position
+// verification), for both layer kinds.
+//
+// ReplaySSM computes every output from the read-only checkpoint and the
+// buffered inputs ("ReplaySSM: Cache SSM Inputs, Not State", Abstract; "ReplaySSM
+// for hybrid SSM-Transformer stacks", How ReplaySSM works, steps 2 and 4).  The
+// prep kernel reduces each (sequence, head)'s buffer to a record
+// (mul_j, z_j, vec_j); this kernel makes the one pass over the checkpoint tile
+//     y_j[r] = mul_j (S0[r, :] . vec_j) + z_j[r],     j < npos, r < R.
+//
+// The pass is bound by HBM bandwidth.  One CTA per SM runs over a contiguous
+// range of tiles with a shared-memory ring of stages; a stage holds a tile and
+// its record.  NT teams of four consumer warps take the tiles in turn (tile k
+// goes to team k mod NT), and each team owns SPT stages of the ring, which it
+// uses in order; one producer thread fills the stages with 1-D bulk copies in
+// tile order (transaction-counted "full" barrier, checkpoint evict-first in
+// L2) and reuses a stage once its team has freed it ("empty" barrier).  Every
+// barrier therefore sees each of its uses waited for in order by the same
+// waiters, so a phase-parity wait never aliases an older phase.  Every wait is
+// bounded: one that gives up sets RS_SEQ_ERR_TIMEOUT and the role stops.
+#include "outputs.cuh"
+#include "launch.h"
+
+namespace rs {
+
+constexpr int kTeamWarps = 4;                   // consumer warps per team (one tile at a time)
+constexpr int kTeamThreads = 32 * kTeamWarps;
+constexpr size_t kStreamSmemBudget = 224 * 1024;
+
+template <int NP>
+struct Roles {
+    static constexpr int NT = NP <= 2 ? 3 : 2;        // consumer teams
+    static constexpr int NCW = NT * kTeamWarps;       // consumer warps
+    static constexpr int THREADS = 32 * (NCW + 1);    // + the producer warp
+};
+
+struct StreamLayout {
+    size_t rec_off, grec_off, stage_bytes, stages, bars, total;
+    int S, SPT;   // stages in all, stages per team
+};
+
+// Stage: tile (padded to 128 bytes) | tile record | group record (Mamba-2).
+__host__ __device__ inline StreamLayout stream_layout(size_t tile_bytes, size_t rec_bytes,
+                                                      size_t grec_bytes, int nt) {
+    StreamLayout l;
+    l.rec_off = align_up(tile_bytes, 128);
+    l.grec_off = align_up(l.rec_off + rec_bytes, 16);
+    l.stage_bytes = align_up(l.grec_off + grec_bytes, 128);
+    size_t spt = (kStreamSmemBudget - 1024) / (l.stage_bytes + 16) / nt;
+    spt = spt < 1 ? 1 : spt > 8 ? 8 : spt;
+    const size_t s = spt * nt;
+    l.S = (int)s;
+    l.SPT = (int)spt;
+    l.stages = 0;
+    l.bars = s * l.stage_bytes;
+    l.total = l.bars + align_up(16 * s, 128);
+    return l;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// 1-D bulk copy without its own expect_tx (the caller sets the total).
+__device__ __forceinline__ void bulk_pieces(void *dst, const void *src, uint32_t bytes,
+                                            uint64_t *bar, uint64_t policy) {
+    uint32_t off = 0;
+    while (off < bytes) {
+        const uint32_t n = bytes - off < 32768u ? bytes - off : 32768u;
+        bulk_g2s(static_cast<char *>(dst) + off, static_cast<const char *>(src) + off, n, bar, policy);
+        off += n;
+    }
+}
+
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+template <int KIND, int CC, typename TS, int NP>
+__global__ void __launch_bounds__(Roles<NP>::THREADS, 1)
+stream_outputs_kernel(const Params p, const void *__restrict__ state, int npos, void *y) {
+    using RL = Roles<NP>;
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int R = p.R, H = p.H;
+    const uint32_t tile_bytes = static_cast<uint32_t>(R) * CC * TS::bytes;
+    const size_t rfl = tile_rec_floats(KIND, NP, R, CC);
+    const size_t gfl = KIND == RS_MAMBA2 ? group_rec_floats(NP, CC) : 0;
+    const uint32_t rec_bytes = static_cast<uint32_t>(4 * rfl), grec_bytes = static_cast<uint32_t>(4 * gfl);
+    const float *trec = p.rec + p.rec_tile_off;
+    const StreamLayout lay = stream_layout(tile_bytes, rec_bytes, grec_bytes, RL::NT);
+    const int S = lay.S, SPT = lay.SPT;
+    // tile k -> team k % NT, the team's m-th tile (m = k / NT), stage
+    // (k % NT) * SPT + m % SPT, use m / SPT of that stage
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.bars);
+    uint64_t *empty = full + S;
+
+    const int ntiles_all = p.B * H;
+    const int per = ntiles_all / gridDim.x, extra = ntiles_all % gridDim.x;
+    const int t0 = blockIdx.x * per + (blockIdx.x < extra ? blockIdx.x : extra);
+    const int nt = per + (blockIdx.x < extra ? 1 : 0);
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, kTeamWarps);
+        }
+    }
+    __syncthreads();
+
+    auto stage = [&](int s) { return smem + lay.stages + (size_t)s * lay.stage_bytes; };
+
+    if (warp == RL::NCW) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            const uint64_t pol_state = policy_evict_first();
+            const uint64_t pol_rec = policy_evict_last();
+            for (int k = 0; k < nt; ++k) {
+                const int m = k / RL::NT, s = (k % RL::NT) * SPT + m % SPT, u = m / SPT;
+                const int tile = t0 + k;
+                if (u >= 1 && !mbar_wait_bounded(empty + s, (u - 1) & 1)) {
+                    atomicOr(&p.err[tile / H], RS_SEQ_ERR_TIMEOUT);
+                    break;
+                }
+                unsigned char *st = stage(s);
+                mbar_expect_tx(full + s, tile_bytes + rec_bytes + grec_bytes);
+                bulk_pieces(st + lay.rec_off, trec + (size_t)tile * rfl, rec_bytes, full + s, pol_rec);
+                if (KIND == RS_MAMBA2) {   // C of the output positions, one record per (sequence, group)
+                    const int b = tile / H, g = (tile - b * H) / p.heads_per_group;
+                    bulk_pieces(st + lay.grec_off, p.rec + ((size_t)b * p.G + g) * gfl, grec_bytes, full + s, pol_rec);
+                }
+                bulk_pieces(st, static_cast<const unsigned char *>(state) + (size_t)tile * tile_bytes,
+                            tile_bytes, full + s, pol_state);
+            }
+        }
+        return;
+    }
+
+    // -------------------------------------------------------------- consumers
+    // Team `team` (four warps) contracts tiles team, team + NT, ...
+    using G = Geom<CC, TS::bytes>;
+    constexpr int VEC = G::VEC, TPR = G::TPR, CPT = G::CPT;
+    const int team = warp / kTeamWarps;
+    const int ttid = threadIdx.x % kTeamThreads;
+    const int tl = ttid % TPR, row0 = ttid / TPR;
+    const size_t y_pos_stride = (size_t)p.B * H * R;
+    // A lane group (TPR lanes) covers RG rows per iteration: all RG x CPT chunks
+    // are loaded first, each row's partial dot goes to its own accumulator, and
+    // the RG partials are reduced across the group by a reduce-scatter, after
+    // which lane pair (2m, 2m+1) of the group holds the full sum of row m.
+    constexpr int RG = TPR == 8 ? 4 : 1;
+    constexpr int GROUPS = kTeamThreads / TPR;   // lane groups per team
+    const int niter = (R + GROUPS * RG - 1) / (GROUPS * RG);
+    for (int m = 0; m * RL::NT + team < nt; ++m) {
+        const int k = m * RL::NT + team, s = team * SPT + m % SPT, u = m / SPT, tile = t0 + k;
+        if (!mbar_wait_bounded(full + s, u & 1)) {
+            if (lane == 0) atomicOr(&p.err[tile / H], RS_SEQ_ERR_TIMEOUT);
+            break;
+        }
+        const unsigned char *st = stage(s);
+        const float *mul = reinterpret_cast<const float *>(st + lay.rec_off);
+        const float *z = mul + 8;
+        const float *vec = KIND == RS_MAMBA2 ? reinterpret_cast<const float *>(st + lay.grec_off) : z + (size_t)NP * R;
+        float v[NP][CPT * VEC];
+#pragma unroll
+        for (int j = 0; j < NP; ++j)
+#pragma unroll
+            for (int c = 0; c < CPT; ++c)
+#pragma unroll
+                for (int e = 0; e < VEC; ++e)
+                    v[j][c * VEC + e] = j < npos ? vec[j * CC + (tl + c * TPR) * VEC + e] : 0.f;
+        float mj[NP];
+#pragma unroll
+        for (int j = 0; j < NP; ++j) mj[j] = j < npos ? mul[j] : 0.f;
+        const size_t y_off = (size_t)tile * R;
+        for (int it = 0; it < niter; ++it) {
+            const int rbase = (it * GROUPS + row0) * RG;   // first row of this group
+            uint4 raw[RG][CPT];
+#pragma unroll
+            for (int r = 0; r < RG; ++r)
+#pragma unroll
+                for (int c = 0; c < CPT; ++c) {
+                    raw[r][c] = make_uint4(0u, 0u, 0u, 0u);
+                    if (rbase + r < R)
+                        raw[r][c] = *reinterpret_cast<const uint4 *>(
+                            st + ((size_t)(rbase + r) * CC + (tl + c * TPR) * VEC) * TS::bytes);
+                }
+            // even / odd columns accumulate in the two halves of packed fp32 FMAs
+            float2 acc2[NP][RG];
+#pragma unroll
+            for (int j = 0; j < NP; ++j)
+#pragma unroll
+                for (int r = 0; r < RG; ++r) acc2[j][r] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int r = 0; r < RG; ++r)
+#pragma unroll
+                for (int c = 0; c < CPT; ++c) {
+                    float f[VEC];
+                    Chunk<TS>::expand(raw[r][c], f);
+#pragma unroll
+                    for (int e = 0; e < VEC; e += 2)
+#pragma unroll
+                        for (int j = 0; j < NP; ++j)
+                            acc2[j][r] = ffma2(make_float2(f[e], f[e + 1]),
+                                               make_float2(v[j][c * VEC + e], v[j][c * VEC + e + 1]), acc2[j][r]);
+                }
+            float acc[NP][RG];
+#pragma unroll
+            for (int j = 0; j < NP; ++j)
+#pragma unroll
+                for (int r = 0; r < RG; ++r) acc[j][r] = acc2[j][r].x + acc2[j][r].y;
+            if constexpr (RG == 4) {
+                const bool hi = tl & 4, b1 = tl & 2;
+                const int row = rbase + (hi ? 2 : 0) + (b1 ? 1 : 0);
+#pragma unroll
+                for (int j = 0; j < NP; ++j) {
+                    // xor 4: keep rows {0,1} (hi = 0) or {2,3} (hi = 1)
+                    const float k0 = (hi ? acc[j][2] : acc[j][0]) + __shfl_xor_sync(0xffffffffu, hi ? acc[j][0] : acc[j][2], 4);
+                    const float k1 = (hi ? acc[j][3] : acc[j][1]) + __shfl_xor_sync(0xffffffffu, hi ? acc[j][1] : acc[j][3], 4);
+                    // xor 2: keep the first (b1 = 0) or second (b1 = 1) of the pair
+                    float t = (b1 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, b1 ? k0 : k1, 2);
+                    t += __shfl_xor_sync(0xffffffffu, t, 1);
+                    if ((tl & 1) == 0 && row < R && j < npos)
+                        st_out(y, y_off + j * y_pos_stride + row, fmaf(mj[j], t, z[j * R + row]), p.out_dtype);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < NP; ++j) {
+                    const float t = row_sum<TPR>(acc[j][0]);
+                    if (tl == 0 && rbase < R && j < npos)
+                        st_out(y, y_off + j * y_pos_stride + rbase, fmaf(mj[j], t, z[j * R + rbase]), p.out_dtype);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty + s);
+    }
+}
+
+static int g_num_sms[64];
+
+static int num_sms() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return 148;
+    if (!g_num_sms[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        g_num_sms[dev] = n > 0 ? n : 148;
+    }
+    return g_num_sms[dev];
+}
+
+static StreamLayout layout_for(const Params &p, int npos) {
+    const int eb = p.copy_dtype == RS_BF16 ? 2 : p.copy_dtype == RS_E4M3 ? 1 : 4;
+    const int NPr = prep_np(npos);
+    const int nt = NPr <= 2 ? Roles<1>::NT : Roles<8>::NT;
+    return stream_layout((size_t)p.R * p.CC * eb, 4 * tile_rec_floats(p.kind, NPr, p.R, p.CC),
+                         p.kind == RS_MAMBA2 ? 4 * group_rec_floats(NPr, p.CC) : 0, nt);
+}
+
+size_t stream_outputs_smem(const Params &p, int npos) { return layout_for(p, npos).total; }
+
+template <int KIND, int CC, typename TS, int NP>
+static cudaError_t launch_stream_t(const Params &p, int npos, void *y, cudaStream_t st) {
+    const void *state = p.copy_dtype == RS_NONE ? static_cast<const void *>(p.master) : p.copy;
+    const StreamLayout lay = layout_for(p, npos);
+    auto k = stream_outputs_kernel<KIND, CC, TS, NP>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total);
+    if (e != cudaSuccess) return e;
+    const int tiles = p.B * p.H;
+    int grid = num_sms();
+    if (grid > tiles) grid = tiles;
+    k<<<grid, Roles<NP>::THREADS, lay.total, st>>>(p, state, npos, y);
+    return cudaGetLastError();
+}
+
+template <int KIND, int CC, typename TS>
+static cudaError_t launch_stream_np(const Params &p, int npos, void *y, cudaStream_t st) {
+    switch (prep_np(npos)) {
+        case 1: return launch_stream_t<KIND, CC, TS, 1>(p, npos, y, st);
+        case 2: return launch_stream_t<KIND, CC, TS, 2>(p, npos, y, st);
+        case 5: return launch_stream_t<KIND, CC, TS, 5>(p, npos, y, st);
+        default: return launch_stream_t<KIND, CC, TS, 8>(p, npos, y, st);
+    }
+}
+
+template <int KIND>
+struct StreamCC {
+    template <int CC>
+    static cudaError_t go(const Params &p, int npos, void *y, cudaStream_t st) {
+        switch (p.copy_dtype) {
+            case RS_BF16: return launch_stream_np<KIND, CC, StBF16>(p, npos, y, st);
+            case RS_E4M3: return launch_stream_np<KIND, CC, StE4M3>(p, npos, y, st);
+            default: return launch_stream_np<KIND, CC, StF32>(p, npos, y, st);
+        }
+    }
+};
+
+// Output-only replay / verification, optionally preceded by the append of T
+// step inputs: the prep kernel (which also performs the append) writes the
+// records, then the streaming pass reads each checkpoint tile once.
+cudaError_t launch_outputs(const Params &p, int npos, int T, const rs_inputs &in, void *y, cudaStream_t st,
+                           cudaEvent_t *ev) {
+    cudaError_t e;
+    if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess) return e;
+    e = launch_prep(p, npos, T, in, st);
+    if (e != cudaSuccess) return e;
+    if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
+    e = cudaErrorInvalidValue;
+    if (p.kind == RS_MAMBA2) {
+        RS_DISPATCH_CC(p.CC, e = StreamCC<RS_MAMBA2>::go, (p, npos, y, st));
+    } else {
+        RS_DISPATCH_CC(p.CC, e = StreamCC<RS_GDN>::go, (p, npos, y, st));
+    }
+    if (e != cudaSuccess) return e;
+    if (ev) e = cudaEventRecord(ev[2], st);
+    return e;
+}
+
+}  // namespace rs

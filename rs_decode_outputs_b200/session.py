@@ -76,6 +76,12 @@ class ReplaySSM:
         L.rs_decode_outputs(self.handle, y, stream)
         return y
 
+    def decode_step(self, inputs, T=1, y=None, stream=None):
+        """Append T inputs and return the outputs at those T positions."""
+        y = self.new_out(None if T == 1 else T) if y is None else y
+        L.rs_decode_step(self.handle, inputs, T, y, stream)
+        return y
+
     def commit(self, min_len=1, mask=None, stream=None):
         L.rs_commit(self.handle, min_len, mask, stream)
 

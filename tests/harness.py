@@ -45,6 +45,22 @@ def rel_err_inf(y, ref):
     return float(np.max(num / den))
 
 
+def rel_err_fro(y, ref):
+    """||y - ref||_F / ||ref||_F over the whole array (one step's outputs)."""
+    y = np.asarray(y, np.float64)
+    ref = np.asarray(ref, np.float64)
+    return float(np.sqrt(np.sum((y - ref) ** 2)) / max(np.sqrt(np.sum(ref ** 2)), 1e-300))
+
+
+def out_err(y, ref, copy_dtype):
+    """The error measure each output-copy tolerance is read on: the largest
+    per-(sequence, head) relative 2-norm error for fp32 and bf16 checkpoints;
+    for the E4M3 copy (3 mantissa bits, so single output vectors of a tile can
+    lose more than the tolerance to rounding alone) the step's whole output in
+    the Frobenius norm."""
+    return rel_err_fro(y, ref) if copy_dtype == rs.RS_E4M3 else rel_err(y, ref)
+
+
 def torch_dtype(code):
     return {rs.RS_F32: torch.float32, rs.RS_BF16: torch.bfloat16}[code]
 
@@ -135,6 +151,54 @@ class GdnCase:
 
     def gpu_pairs(self, y):
         return f64(y)[..., self.pb, self.ph, :]
+
+
+# ----------------------------------------------- quantised checkpoints ----
+
+def dequantised(S, copy_dtype):
+    """What a kernel reading the low-precision copy of fp32 master S sees, in
+    fp64: bf16 RNE, or E4M3 codes x the per-tile scale (absmax / 448)."""
+    S32 = np.asarray(S, np.float64).astype(np.float32)
+    if copy_dtype == rs.RS_BF16:
+        return oracle.bf16_decode(oracle.bf16_rne(S32)).astype(np.float64)
+    if copy_dtype == rs.RS_E4M3:
+        out = np.empty(S32.shape, np.float64)
+        for i in range(S32.shape[0]):
+            codes, scale = oracle.e4m3_quantize_tile(S32[i])
+            out[i] = oracle.e4m3_decode(codes).astype(np.float64) * np.float64(np.float32(scale))
+        return out
+    return S32.astype(np.float64)
+
+
+class QuantCheckpoint:
+    """Oracle bookkeeping of the method's checkpoint for a low-precision arm.
+
+    Outputs are replayed from the dequantised copy of the checkpoint plus the
+    inputs buffered since it ("ReplaySSM: Cache SSM Inputs, Not State",
+    Abstract: outputs come from the checkpoint and the cached inputs).  A
+    commit of the dual-precision arm folds the buffer into the fp64 checkpoint;
+    the shared arm has no master, so its commit folds the buffer into the
+    dequantised copy, which is then quantised again."""
+
+    def __init__(self, case, copy_dtype, shared):
+        self.case, self.copy_dtype, self.shared = case, copy_dtype, shared
+        self.ckpt = case.hstate.copy()
+        self.buf = []
+
+    def _cat(self):
+        return {k: torch.cat([d[k] for d in self.buf], 0) for k in self.buf[0]}
+
+    def step(self, s):
+        """Appends step s; returns its expected outputs [T_s, n, R]."""
+        self.buf.append(s)
+        T = next(iter(s.values())).shape[0]
+        y, _ = self.case.oracle_run(self._cat(), h=dequantised(self.ckpt, self.copy_dtype))
+        return y[-T:]
+
+    def commit(self):
+        start = dequantised(self.ckpt, self.copy_dtype) if self.shared else self.ckpt
+        _, self.ckpt = self.case.oracle_run(self._cat(), h=start)
+        self.buf = []
 
 
 # -------------------------------------------------------------- checks ----

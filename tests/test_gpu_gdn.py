@@ -8,12 +8,12 @@ import oracle
 import rs_decode_outputs_b200 as rs
 from oracle.replay_model import RingPointers
 from tests.harness import (TOL_BF16, TOL_E4M3, TOL_F32, GdnCase, check_copy_is_quantised_master,
-                           make_session, rel_err)
+                           make_session, out_err, rel_err)
 
 pytestmark = pytest.mark.gpu
 
 
-def decode_run(case, sess, steps, K, check_drift=False):
+def decode_run(case, sess, steps, K, check_drift=False, errs=None):
     ptr = RingPointers(case.B, sess.cfg.cap)
     worst = 0.0
     for t in range(steps):
@@ -22,7 +22,10 @@ def decode_run(case, sess, steps, K, check_drift=False):
         ptr.append(1)
         y = sess.decode()
         ref, _ = case.oracle_run(s)
-        worst = max(worst, rel_err(case.gpu_pairs(y), ref[0]))
+        e = out_err(case.gpu_pairs(y), ref[0], sess.cfg.copy_dtype)
+        worst = max(worst, e)
+        if errs is not None:
+            errs.append(e)
         if ptr.length[0] >= K:
             sess.commit(min_len=K)
             ptr.commit(min_len=K)
@@ -113,10 +116,11 @@ def test_eager_baseline_kernel(cuda_device, sdt, tol):
 def test_shared_lowp_arm_runs_and_is_not_better(cuda_device):
     """The comparison arm (one shared low-precision checkpoint that also serves
     the updates) against the dual-precision arm, both E4M3, from the same
-    prefilled checkpoint: the dual arm stays within the fp8 tolerance and is
-    no worse than the shared arm."""
+    prefilled checkpoint: the dual arm stays within the fp8 tolerance, and on
+    average over the run it is closer to the fp64 truth than the shared arm,
+    whose every commit quantises again."""
     B, H, dk, dv, K = 2, 4, 64, 64, 4
-    errs = {}
+    worst, mean = {}, {}
     for shared in (0, 1):
         case = GdnCase(B, H, dk, dv, rs.RS_BF16, seed=161, device=cuda_device)
         sess = make_session(rs.RS_GDN, B, H, dv, dk, cap=8, copy_dtype=rs.RS_E4M3,
@@ -126,6 +130,8 @@ def test_shared_lowp_arm_runs_and_is_not_better(cuda_device):
         sess.eager_step(state, rs.RS_F32, pre, 64)
         case.oracle_run(pre)
         sess.load_checkpoint(state)
-        errs[shared] = decode_run(case, sess, 64, K=K)
-    assert errs[0] <= TOL_E4M3, errs
-    assert errs[0] <= errs[1] * 1.05, errs
+        errs = []
+        worst[shared] = decode_run(case, sess, 64, K=K, errs=errs)
+        mean[shared] = float(np.mean(errs))
+    assert worst[0] <= TOL_E4M3, worst
+    assert mean[0] < mean[1], mean

@@ -7,12 +7,12 @@ import torch
 import rs_decode_outputs_b200 as rs
 from oracle.replay_model import RingPointers
 from tests.harness import (TOL_BF16, TOL_E4M3, TOL_F32, Mamba2Case, check_copy_is_quantised_master,
-                           make_session, rel_err)
+                           make_session, out_err, rel_err)
 
 pytestmark = pytest.mark.gpu
 
 
-def decode_run(case, sess, steps, K, check_ptrs=True, check_drift=False):
+def decode_run(case, sess, steps, K, check_ptrs=True, check_drift=False, errs=None):
     """Append / decode / commit-at-K loop; returns the max relative error."""
     ptr = RingPointers(case.B, sess.cfg.cap)
     worst = 0.0
@@ -22,7 +22,10 @@ def decode_run(case, sess, steps, K, check_ptrs=True, check_drift=False):
         ptr.append(1)
         y = sess.decode()
         ref, _ = case.oracle_run(s)
-        worst = max(worst, rel_err(case.gpu_pairs(y), ref[0]))
+        e = out_err(case.gpu_pairs(y), ref[0], sess.cfg.copy_dtype)
+        worst = max(worst, e)
+        if errs is not None:
+            errs.append(e)
         if ptr.length[0] >= K:
             sess.commit(min_len=K)
             ptr.commit(min_len=K)
