@@ -94,7 +94,10 @@ typedef struct {
 /* Step inputs.  Mamba-2 uses x, dt, B, C; GDN uses q, k, v, alpha, beta.
  * dt, alpha, beta are fp32; the others are in_dtype.  Shapes for T steps:
  *   x [T][B][H][P]   dt [T][B][H]   B, C [T][B][G][N]      (dt after softplus)
- *   q, k [T][B][H][dk]   v [T][B][H][dv]   alpha, beta [T][B][H]              */
+ *   q, k [T][B][H][dk]   v [T][B][H][dv]   alpha, beta [T][B][H]
+ * Device memory, contiguous, naturally aligned (fp32 arrays to 4 bytes, bf16 to
+ * 2); Mamba-2's B and C must be 16-byte aligned.  A missing or misaligned
+ * pointer makes the call return RS_ERR_ARG.                                   */
 typedef struct {
     const void *x;
     const float *dt;
@@ -128,8 +131,8 @@ typedef struct {
     size_t scratch, scratch_bytes; /* fp32 replay records, written and read inside one
                                       output call (NP = npos_max rounded up to 1, 2, 5, 8):
                                       Mamba-2: [B][G][NP Cc] group records, then
-                                      [B][H][8 + NP R] tile records; GDN: [B][H][8 + NP (R
-                                      + Cc)]; each record rounded up to 16 bytes          */
+                                      [B][H][16 + NP cap] tile records; GDN: [B][H][16 +
+                                      NP (cap + Cc)]; each record rounded up to 16 bytes  */
     size_t total;
 } rs_layout;
 

@@ -106,15 +106,24 @@ rs_status make_layout(const rs_config *c, rs_layout *L) {
     put(L->err, dummy, 4 * B);
     put(L->arrive, dummy, 4 * B);
     put(L->scratch, L->scratch_bytes,
-        4 * rs::scratch_floats(c->kind, c->batch, c->nheads, c->ngroups, c->npos_max, c->headdim, c->dstate));
+        4 * rs::scratch_floats(c->kind, c->batch, c->nheads, c->ngroups, c->npos_max, c->cap, c->dstate));
     L->total = o;
     return RS_OK;
 }
 
-bool has_inputs(int kind, const rs_inputs *in) {
+bool aligned(const void *ptr, uintptr_t n) { return (reinterpret_cast<uintptr_t>(ptr) & (n - 1)) == 0; }
+
+// All inputs of the layer kind present and aligned: fp32 arrays to 4 bytes,
+// activations to their element size, and Mamba-2's B and C to 16 bytes (their
+// rows are read in 16-byte pieces).
+bool has_inputs(int kind, int in_dtype, const rs_inputs *in) {
     if (!in) return false;
-    if (kind == RS_MAMBA2) return in->x && in->dt && in->B && in->C;
-    return in->q && in->k && in->v && in->alpha && in->beta;
+    const uintptr_t eb = in_dtype == RS_BF16 ? 2 : 4;
+    if (kind == RS_MAMBA2)
+        return in->x && in->dt && in->B && in->C && aligned(in->x, eb) && aligned(in->dt, 4) &&
+               aligned(in->B, 16) && aligned(in->C, 16);
+    return in->q && in->k && in->v && in->alpha && in->beta && aligned(in->q, eb) && aligned(in->k, eb) &&
+           aligned(in->v, eb) && aligned(in->alpha, 4) && aligned(in->beta, 4);
 }
 
 }  // namespace
@@ -296,7 +305,7 @@ rs_status rs_load_checkpoint(rs_handle h, const float *state, rs_stream stream) 
 }
 
 rs_status rs_append(rs_handle h, const rs_inputs *in, int T, rs_stream stream) {
-    if (!h || !has_inputs(h->cfg.kind, in)) return RS_ERR_ARG;
+    if (!h || !has_inputs(h->cfg.kind, h->cfg.in_dtype, in)) return RS_ERR_ARG;
     if (T < 1) return RS_ERR_ARG;
     if (T > h->cfg.cap) return RS_ERR_CAPACITY;
     return launched(rs::launch_append(h->p, *in, T, static_cast<cudaStream_t>(stream)), "append");
@@ -314,7 +323,7 @@ rs_status rs_decode_outputs(rs_handle h, void *y, rs_stream stream) {
 }
 
 rs_status rs_decode_step(rs_handle h, const rs_inputs *in, int T, void *y, rs_stream stream) {
-    if (!h || !y || !has_inputs(h->cfg.kind, in)) return RS_ERR_ARG;
+    if (!h || !y || !has_inputs(h->cfg.kind, h->cfg.in_dtype, in)) return RS_ERR_ARG;
     if (T < 1) return RS_ERR_ARG;
     if (T > h->cfg.npos_max || T > h->cfg.cap) return RS_ERR_CAPACITY;
     return launched(rs::launch_outputs(h->p, T, T, *in, y, static_cast<cudaStream_t>(stream), prof_slot(h)),
@@ -341,7 +350,7 @@ rs_status rs_rollback(rs_handle h, const int32_t *k, rs_stream stream) {
 
 static rs_status eager(rs_handle h, void *state, int sdt, const rs_inputs *in, int T, void *y,
                        const int32_t *cur, int nslots, rs_stream stream) {
-    if (!h || !state || !y || !has_inputs(h->cfg.kind, in) || T < 1) return RS_ERR_ARG;
+    if (!h || !state || !y || !has_inputs(h->cfg.kind, h->cfg.in_dtype, in) || T < 1) return RS_ERR_ARG;
     if (sdt != RS_F32 && sdt != RS_BF16) return RS_ERR_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (h->cfg.kind == RS_MAMBA2)

@@ -1,32 +1,34 @@
 // Replay prologue ("prep") kernels, optionally fused with the append of the
 // step's inputs.
 //
-// For every (sequence, head) they reduce the buffered inputs to the few
-// numbers the output-only pass needs at NP output positions (e_j = L - npos + j,
-// 0-based buffer index), so that  y_j[r] = mul_j (S0[r, :] . vec_j) + z_j[r]:
+// For every (sequence, head) they reduce the buffer to the few numbers the
+// streaming pass needs at NP output positions e_j = L - npos + j (0-based
+// buffer index), so that
+//     y_j[r] = mul_j (S0[r, :] . vec_j) + sum_{i<=e_j} coef_j[i] w_i[r]
+// with w_i the head's ring row of entry i, which the streaming pass reads
+// together with the checkpoint tile.
 // Mamba-2 ("ReplaySSM for hybrid SSM-Transformer stacks", How ReplaySSM works,
 // step 2: the output is a function of the checkpoint and the recent inputs):
 //   vec_j = C_{e_j},  mul_j = exp(A sum_{m<=e_j} dt_m) (x the fp8 tile scale),
-//   z_j = sum_{i<=e_j} exp(A sum_{i<m<=e_j} dt_m) dt_i (B_i . C_{e_j}) x_i + D x_{e_j}
+//   coef_j[i] = exp(A sum_{i<m<=e_j} dt_m) dt_i (B_i . C_{e_j})  (+ D at i = e_j),
+//   w_i = x_i.
 // GDN:  vec_j = M_1..M_{e_j} q_{e_j}  (M_i = alpha_i (I - beta_i k_i k_i^T)), by the
 //   backward sweep  u <- q_{e_j};  for i = e_j..1: c_i = beta_i (k_i . u);
-//   u <- alpha_i (u - c_i k_i);  mul_j = scale (x tile scale),  z_j = scale sum_i c_i v_i.
+//   u <- alpha_i (u - c_i k_i);  mul_j = scale (x tile scale),
+//   coef_j[i] = scale c_i,  w_i = v_i.
 //
 // With T > 0 the kernel also appends the T step inputs (step 2: append the new
-// SSM input to the buffer): the new entries are read straight from the inputs,
-// written into their ring slots, and the last CTA of a sequence to finish
-// advances its tail by T (per-sequence arrival counter).  A sequence whose
-// buffer would overflow is left unchanged and flagged.
-//
-// Both kernels are short latency-bound chains; they read the pointers once,
-// stage exactly the buffered rows they need into shared memory with one round
-// of asynchronous copies, and compute from shared memory.
+// SSM input to the buffer): the new entries are read straight from the inputs
+// and written into their ring slots, and the last CTA of a sequence to finish
+// advances its tail by T (per-sequence arrival counter; every CTA has read the
+// pointers before it arrives).  A sequence whose buffer would overflow is left
+// unchanged and flagged.
 #include "outputs.cuh"
 #include "launch.h"
 
 namespace rs {
 
-constexpr int kPrepWarps = 8;   // warps per CTA, one head per warp
+constexpr int kPrepWarps = 8;   // warps per CTA
 
 __device__ __forceinline__ float warp_incl_scan(float v, int lane) {
 #pragma unroll
@@ -66,7 +68,7 @@ __device__ __forceinline__ void copy_row(void *dst, const void *src, int bytes, 
     }
 }
 
-// Last arrival of the CTAs of sequence b advances its tail by T.
+// Last arrival of the `ctas` CTAs of sequence b advances its tail by T.
 __device__ __forceinline__ void arrive_and_advance(const Params &p, int b, int tail, int T, int ctas) {
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -78,225 +80,260 @@ __device__ __forceinline__ void arrive_and_advance(const Params &p, int b, int t
     }
 }
 
-// ---------------------------------------------------------------- Mamba-2 --
-// One CTA per (sequence, group, chunk of kPrepWarps heads).  Buffered entries
-// are staged compactly, buffer index i at row i.  Shared memory:
-//   braw [cap][CC] | craw [NP][CC] | Cf [NP][CC] | bc [NP][cap] |
-//   per warp: xraw [cap][R] | dt [cap] | cum [cap] | coef [NP][cap]
-struct M2PrepSmem {
-    size_t braw, craw, cf, bc, warps, per_warp, x, dt, cum, coef, total;
-};
+__device__ __forceinline__ void write_header(float *trec, int head, int L, int cap_mask) {
+    trec[kRecHeadSlot] = __int_as_float(head & cap_mask);
+    trec[kRecLen] = __int_as_float(L);
+}
 
-__host__ __device__ inline M2PrepSmem m2_prep_smem(int cap, int R, int CC, int NP, int ib) {
-    M2PrepSmem s;
-    size_t o = 0;
-    s.braw = o; o = align_up(o + (size_t)cap * CC * ib, 16);
-    s.craw = o; o = align_up(o + (size_t)NP * CC * ib, 16);
-    s.cf = o;   o = align_up(o + 4 * (size_t)NP * CC, 16);
-    s.bc = o;   o = align_up(o + 4 * (size_t)NP * cap, 16);
-    s.warps = o;
-    size_t w = 0;
-    s.x = w;    w = align_up(w + (size_t)cap * R * ib, 16);
-    s.dt = w;   w = align_up(w + 4 * (size_t)cap, 16);
-    s.cum = w;  w = align_up(w + 4 * (size_t)cap, 16);
-    s.coef = w; w = align_up(w + 4 * (size_t)NP * cap, 16);
-    s.per_warp = w;
-    s.total = o + kPrepWarps * w;
-    return s;
+// Sum of the elementwise products of two 16-byte chunks of bf16 or fp32.
+__device__ __forceinline__ float chunk_dot(const uint4 &a, const uint4 &c, int ib) {
+    if (ib == 2) {
+        float d = bf16_lo(a.x) * bf16_lo(c.x);
+        d = fmaf(bf16_hi(a.x), bf16_hi(c.x), d);
+        d = fmaf(bf16_lo(a.y), bf16_lo(c.y), d);
+        d = fmaf(bf16_hi(a.y), bf16_hi(c.y), d);
+        d = fmaf(bf16_lo(a.z), bf16_lo(c.z), d);
+        d = fmaf(bf16_hi(a.z), bf16_hi(c.z), d);
+        d = fmaf(bf16_lo(a.w), bf16_lo(c.w), d);
+        return fmaf(bf16_hi(a.w), bf16_hi(c.w), d);
+    }
+    float d = __uint_as_float(a.x) * __uint_as_float(c.x);
+    d = fmaf(__uint_as_float(a.y), __uint_as_float(c.y), d);
+    d = fmaf(__uint_as_float(a.z), __uint_as_float(c.z), d);
+    return fmaf(__uint_as_float(a.w), __uint_as_float(c.w), d);
+}
+
+// ---------------------------------------------------------------- Mamba-2 --
+// One CTA per (sequence, group).  Every global read is issued in bulk, with
+// no dependence between threads: the group's B_i . C_{e_j} are formed once
+// (lane groups of TPRB lanes per B row, the rows spread over the warps), and
+// dt of a chunk of up to kM2HeadChunk heads is staged for all entries at once;
+// then each warp takes heads of the chunk in turn (prefix sums of dt,
+// multipliers, coefficients) from shared memory, writing the head's record.
+// Shared memory: bc [NP][cap] | dt [HC][cap] | per warp: cum [cap].
+constexpr int kM2StageFloats = 4096;   // dt floats staged per round
+
+__host__ __device__ inline int m2_head_chunk(int hpg, int cap) {
+    const int hc = kM2StageFloats / cap;
+    return hc < 1 ? 1 : hc < hpg ? hc : hpg;
+}
+
+__host__ __device__ inline size_t m2_prep_floats(int cap, int NP, int hpg) {
+    return (size_t)NP * cap + (size_t)m2_head_chunk(hpg, cap) * cap + (size_t)kPrepWarps * cap;
+}
+
+// Copy `rows` rows of `row_bytes` bytes from a contiguous source to
+// dst0 + r * dst_stride with every thread of the CTA, loads issued ahead of
+// the stores; 16-, 4- or 2-byte units as the addresses allow.
+__device__ __forceinline__ void copy_rows_cta(unsigned char *dst0, size_t dst_stride, const unsigned char *src,
+                                              int rows, int row_bytes) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(dst0) | (uintptr_t)dst_stride |
+                        reinterpret_cast<uintptr_t>(src) | (uintptr_t)row_bytes;
+    const int unit = (a & 15) == 0 ? 16 : (a & 3) == 0 ? 4 : 2;
+    const int upr = row_bytes / unit, total = rows * upr;
+    constexpr int U = 4;
+    for (int k0 = threadIdx.x; k0 < total; k0 += U * blockDim.x) {
+        uint4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int k = k0 + u * blockDim.x;
+            if (k >= total) break;
+            const unsigned char *s = src + (size_t)k * unit;
+            if (unit == 16) v[u] = *reinterpret_cast<const uint4 *>(s);
+            else if (unit == 4) v[u].x = *reinterpret_cast<const uint32_t *>(s);
+            else v[u].x = *reinterpret_cast<const uint16_t *>(s);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int k = k0 + u * blockDim.x;
+            if (k >= total) break;
+            const int r = k / upr, w = k - (k / upr) * upr;
+            unsigned char *d = dst0 + (size_t)r * dst_stride + (size_t)w * unit;
+            if (unit == 16) *reinterpret_cast<uint4 *>(d) = v[u];
+            else if (unit == 4) *reinterpret_cast<uint32_t *>(d) = v[u].x;
+            else *reinterpret_cast<uint16_t *>(d) = static_cast<uint16_t>(v[u].x);
+        }
+    }
 }
 
 template <int CC, int NP>
 __global__ void __launch_bounds__(32 * kPrepWarps)
 m2_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
-    extern __shared__ __align__(16) unsigned char psm[];
-    __shared__ int s_head, s_tail;
+    extern __shared__ __align__(16) float psm[];
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int Bn = p.B, H = p.H, R = p.R, cap = p.cap, ib = p.in_dtype == RS_BF16 ? 2 : 4;
-    const int hpg = p.heads_per_group;
-    const int g = blockIdx.y, b = blockIdx.z;
-    const int hl = blockIdx.x * kPrepWarps + warp;   // head within the group
-    const bool has_head = hl < hpg;
-    const int h = g * hpg + hl;
-    const int tile = b * H + h;
-    const M2PrepSmem S = m2_prep_smem(cap, R, CC, NP, ib);
-    unsigned char *braw = psm + S.braw, *craw = psm + S.craw;
-    float *Cf = reinterpret_cast<float *>(psm + S.cf), *bc = reinterpret_cast<float *>(psm + S.bc);
-    unsigned char *wsm = psm + S.warps + (size_t)warp * S.per_warp;
-    unsigned char *xraw = wsm + S.x;
-    float *dt = reinterpret_cast<float *>(wsm + S.dt), *cum = reinterpret_cast<float *>(wsm + S.cum);
-    float *coef = reinterpret_cast<float *>(wsm + S.coef);
-    const size_t trf = tile_rec_floats(RS_MAMBA2, NP, R, CC);
-    float *trec = p.rec + p.rec_tile_off + (size_t)tile * trf;
-    float *grec = p.rec + ((size_t)b * p.G + g) * group_rec_floats(NP, CC);
-    const size_t rowB = (size_t)CC * ib, rowX = (size_t)R * ib;
+    const int Bn = p.B, H = p.H, R = p.R, cap = p.cap, G = p.G, hpg = p.heads_per_group;
+    const int ib = p.in_dtype == RS_BF16 ? 2 : 4;
+    const int b = blockIdx.x / G, g = blockIdx.x - (blockIdx.x / G) * G;
+    const int HC = m2_head_chunk(hpg, cap);
+    float *bc = psm;
+    float *sdt = psm + (size_t)NP * cap;
+    float *cum = sdt + (size_t)HC * cap + (size_t)warp * cap;
+    const size_t trf = tile_rec_floats(RS_MAMBA2, NP, cap, CC);
+    float *grec = p.rec + ((size_t)b * G + g) * group_rec_floats(NP, CC);
+    float *trec0 = p.rec + p.rec_tile_off + ((size_t)b * H + (size_t)g * hpg) * trf;   // the group's heads
+    const int h0 = g * hpg;   // first head of the group
 
-    if (threadIdx.x == 0) {
-        s_head = p.head[b];
-        s_tail = p.tail[b];
-    }
-    __syncthreads();
-    const int head = s_head, tail = s_tail, L_old = tail - head, L = L_old + T;
+    const int head = p.head[b], tail = p.tail[b];
+    const int L_old = tail - head, L = L_old + T;
     if (L_old < 0 || L > cap) {   // corrupt pointers or ring overflow: nothing is appended
-        if (has_head)
-            for (size_t i = lane; i < trf; i += 32) trec[i] = 0.f;
-        if (blockIdx.x == 0)
-            for (size_t i = threadIdx.x; i < (size_t)NP * CC; i += blockDim.x) grec[i] = 0.f;
-        if (threadIdx.x == 0) atomicOr(&p.err[b], T > 0 ? RS_SEQ_ERR_OVERFLOW : RS_SEQ_ERR_EMPTY);
+        for (size_t i = threadIdx.x; i < (size_t)hpg * trf; i += blockDim.x) trec0[i] = 0.f;
+        for (int i = threadIdx.x; i < NP * CC; i += blockDim.x) grec[i] = 0.f;
+        if (g == 0 && threadIdx.x == 0) atomicOr(&p.err[b], T > 0 ? RS_SEQ_ERR_OVERFLOW : RS_SEQ_ERR_EMPTY);
         return;
     }
-    const bool ok = npos >= 1 && L >= npos;
-    const unsigned char *bblk = static_cast<const unsigned char *>(p.rc) + ((size_t)b * p.G + g) * p.blk_c;
-    const unsigned char *cblk = static_cast<const unsigned char *>(p.rd) + ((size_t)b * p.G + g) * p.blk_c;
-    const unsigned char *xblk = static_cast<const unsigned char *>(p.ra) + (size_t)tile * p.blk_r;
-    const float *dtblk = static_cast<const float *>(p.rb) + (size_t)tile * p.capd;
-    // source row of buffer entry i: ring slot for the entries already buffered, the step inputs for the new ones
-    auto b_src = [&](int i) -> const void * {
-        return i < L_old ? static_cast<const void *>(bblk + (size_t)((head + i) & p.cap_mask) * rowB)
-                         : static_cast<const void *>(static_cast<const unsigned char *>(in.B) +
-                                                     (((size_t)(i - L_old) * Bn + b) * p.G + g) * rowB);
+    const size_t rowB = (size_t)CC * ib, rowX = (size_t)R * ib;
+    unsigned char *bblk = static_cast<unsigned char *>(p.rc) + ((size_t)b * G + g) * p.blk_c;
+    unsigned char *cblk = static_cast<unsigned char *>(p.rd) + ((size_t)b * G + g) * p.blk_c;
+    const float *dtring = static_cast<const float *>(p.rb) + ((size_t)b * H + h0) * p.capd;   // [hpg][capd]
+    // row of buffer entry i: its ring slot for the entries already buffered, the step inputs for the new ones
+    auto b_row = [&](int i) -> const unsigned char * {
+        return i < L_old ? bblk + (size_t)((head + i) & p.cap_mask) * rowB
+                         : static_cast<const unsigned char *>(in.B) + (((size_t)(i - L_old) * Bn + b) * G + g) * rowB;
     };
-    auto c_src = [&](int i) -> const void * {
-        return i < L_old ? static_cast<const void *>(cblk + (size_t)((head + i) & p.cap_mask) * rowB)
-                         : static_cast<const void *>(static_cast<const unsigned char *>(in.C) +
-                                                     (((size_t)(i - L_old) * Bn + b) * p.G + g) * rowB);
+    auto c_row = [&](int i) -> const unsigned char * {
+        return i < L_old ? cblk + (size_t)((head + i) & p.cap_mask) * rowB
+                         : static_cast<const unsigned char *>(in.C) + (((size_t)(i - L_old) * Bn + b) * G + g) * rowB;
     };
-    // ---- one round of asynchronous copies
-    if (ok) {
-        for (int i = warp; i < L; i += kPrepWarps) stage_row(braw + (size_t)i * rowB, b_src(i), (int)rowB, lane, 32);
-        for (int j = warp; j < npos; j += kPrepWarps)
-            stage_row(craw + (size_t)j * rowB, c_src(L - npos + j), (int)rowB, lane, 32);
-    }
-    if (has_head) {
-        for (int i = 0; i < L; ++i) {
-            const void *src = i < L_old ? static_cast<const void *>(xblk + (size_t)((head + i) & p.cap_mask) * rowX)
-                                        : static_cast<const void *>(static_cast<const unsigned char *>(in.x) +
-                                                                    (((size_t)(i - L_old) * Bn + b) * H + h) * rowX);
-            stage_row(xraw + (size_t)i * rowX, src, (int)rowX, lane, 32);
-        }
-        for (int i = lane; i < L; i += 32)
-            cp_async4(dt + i, i < L_old ? dtblk + ((head + i) & p.cap_mask) : in.dt + ((size_t)(i - L_old) * Bn + b) * H + h);
-    }
-    cp_async_wait_all();
-    __syncthreads();
+    auto dt_at = [&](int hl, int i) -> float {
+        return i < L_old ? dtring[(size_t)hl * p.capd + ((head + i) & p.cap_mask)]
+                         : in.dt[((size_t)(i - L_old) * Bn + b) * H + h0 + hl];
+    };
 
+    const bool ok = npos >= 1 && L >= npos;
     if (ok) {
-        // ---- C of the output positions as fp32, and B_i . C_{e_j} (shared by the CTA's heads)
-        for (int q = threadIdx.x; q < npos * CC; q += blockDim.x) Cf[q] = lds_in(craw, q, p.in_dtype);
-        __syncthreads();
-        if (blockIdx.x == 0)
-            for (int q = threadIdx.x; q < npos * CC; q += blockDim.x) grec[q] = Cf[q];
-        for (int w = warp; w < npos * L; w += kPrepWarps) {
-            const int j = w / L, i = w - (w / L) * L;
-            if (i > L - npos + j) continue;
-            float d = 0.f;
-            for (int n = lane; n < CC; n += 32) d = fmaf(lds_in(braw, (size_t)i * CC + n, p.in_dtype), Cf[j * CC + n], d);
-            d = warp_sum(d);
-            if (lane == 0) bc[j * cap + i] = d;
+        // ---- B_i . C_{e_j} for i < L (and the group record: C_{e_j} in fp32)
+        const int nch = CC * ib / 16;
+        const int TPRB = nch < 32 ? nch : 32, CPLB = nch / TPRB, RPI = 32 / TPRB;
+        const int q = lane % TPRB, sub = lane / TPRB;
+        uint4 cch[NP][2];
+#pragma unroll
+        for (int j = 0; j < NP; ++j)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                cch[j][c] = make_uint4(0u, 0u, 0u, 0u);
+                if (j < npos && c < CPLB)
+                    cch[j][c] = reinterpret_cast<const uint4 *>(c_row(L - npos + j))[q + c * TPRB];
+            }
+        if (warp == 0 && sub == 0) {
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+                if (j >= npos) break;
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    if (c >= CPLB) break;
+                    const int col = (q + c * TPRB) * (16 / ib);
+                    const uint4 w = cch[j][c];
+                    if (ib == 2) {
+                        float4 *dst = reinterpret_cast<float4 *>(grec + j * CC + col);
+                        dst[0] = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
+                        dst[1] = make_float4(bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w));
+                    } else {
+                        *reinterpret_cast<uint4 *>(grec + j * CC + col) = w;
+                    }
+                }
+            }
         }
-        __syncthreads();
-        if (has_head) {
-            // ---- per head: prefix sums of dt, coefficients, z
-            float *mul = trec, *z = trec + 8;
-            const float A = p.A[h];
-            const float Dh = p.D ? p.D[h] : 0.f;
-            const float tscale = p.copy_dtype == RS_E4M3 ? p.scale[tile] : 1.f;
-            float carry = 0.f;
-            for (int i0 = 0; i0 < L; i0 += 32) {
-                const int i = i0 + lane;
-                const float d = i < L ? dt[i] : 0.f;
-                const float c = warp_incl_scan(d, lane) + carry;
-                if (i < L) cum[i] = c;
-                carry = __shfl_sync(0xffffffffu, c, 31);
-            }
-            __syncwarp();
-            for (int j = 0; j < npos; ++j) {
-                const int e = L - npos + j;
-                const float ce = cum[e];
-                if (lane == 0) mul[j] = expf(A * ce) * tscale;
-                for (int i = lane; i <= e; i += 32) coef[j * cap + i] = expf(A * (ce - cum[i])) * dt[i] * bc[j * cap + i];
-            }
-            __syncwarp();
-            constexpr int RL = 8;   // rows per lane, R <= 256
-            float acc[NP][RL];
+        for (int i0 = warp * RPI; i0 < L; i0 += kPrepWarps * RPI) {
+            const int i = i0 + sub;
+            uint4 bch[2];
 #pragma unroll
-            for (int j = 0; j < NP; ++j)
+            for (int c = 0; c < 2; ++c) {
+                bch[c] = make_uint4(0u, 0u, 0u, 0u);
+                if (i < L && c < CPLB) bch[c] = reinterpret_cast<const uint4 *>(b_row(i))[q + c * TPRB];
+            }
 #pragma unroll
-                for (int m = 0; m < RL; ++m) acc[j][m] = 0.f;
-            for (int i = 0; i < L; ++i) {
-                float cf[NP];
+            for (int j = 0; j < NP; ++j) {
+                if (j >= npos) break;
+                float d = chunk_dot(bch[0], cch[j][0], ib);
+                if (CPLB > 1) d += chunk_dot(bch[1], cch[j][1], ib);
+                for (int o = TPRB / 2; o >= 1; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+                if (q == 0 && i < L) bc[j * cap + i] = d;
+            }
+        }
+        const bool tscale_on = p.copy_dtype == RS_E4M3;
+        for (int c0 = 0; c0 < hpg; c0 += HC) {
+            const int nh = hpg - c0 < HC ? hpg - c0 : HC;
+            // ---- dt of the chunk's heads, all entries at once
+            for (int k = threadIdx.x; k < nh * L; k += blockDim.x) {
+                const int hl = k / L, i = k - (k / L) * L;
+                sdt[hl * cap + i] = dt_at(c0 + hl, i);
+            }
+            __syncthreads();
+            // ---- per head: prefix sums of dt, multipliers, coefficients
+            for (int hc = warp; hc < nh; hc += kPrepWarps) {
+                const int hl = c0 + hc, h = h0 + hl;
+                const float *dts = sdt + (size_t)hc * cap;
+                float *trec = trec0 + (size_t)hl * trf;
+                float carry = 0.f;
+                for (int i0 = 0; i0 < L; i0 += 32) {
+                    const int i = i0 + lane;
+                    const float c = warp_incl_scan(i < L ? dts[i] : 0.f, lane) + carry;
+                    if (i < L) cum[i] = c;
+                    carry = __shfl_sync(0xffffffffu, c, 31);
+                }
+                __syncwarp();
+                const float A = p.A[h];
+                const float Dh = p.D ? p.D[h] : 0.f;
+                const float tscale = tscale_on ? p.scale[(size_t)b * H + h] : 1.f;
 #pragma unroll
                 for (int j = 0; j < NP; ++j) {
+                    if (j >= npos) break;
                     const int e = L - npos + j;
-                    cf[j] = (j < npos && i <= e) ? coef[j * cap + i] : 0.f;
-                    if (j < npos && i == e) cf[j] += Dh;
+                    const float ce = cum[e];
+                    if (lane == 0) trec[j] = expf(A * ce) * tscale;
+                    float *coef = trec + kRecHdr + (size_t)j * cap;
+                    for (int i = lane; i < L; i += 32)
+                        coef[i] = i <= e ? fmaf(expf(A * (ce - cum[i])) * dts[i], bc[j * cap + i], i == e ? Dh : 0.f)
+                                         : 0.f;
                 }
-#pragma unroll
-                for (int m = 0; m < RL; ++m) {
-                    const int r = lane + 32 * m;
-                    if (r >= R) break;
-                    const float xv = lds_in(xraw, (size_t)i * R + r, p.in_dtype);
-#pragma unroll
-                    for (int j = 0; j < NP; ++j) acc[j][m] = fmaf(cf[j], xv, acc[j][m]);
-                }
+                if (lane == 0) write_header(trec, head, L, p.cap_mask);
+                __syncwarp();   // cum is reused by the warp's next head
             }
-#pragma unroll
-            for (int m = 0; m < RL; ++m) {
-                const int r = lane + 32 * m;
-                if (r >= R) break;
-#pragma unroll
-                for (int j = 0; j < NP; ++j)
-                    if (j < npos) z[j * R + r] = acc[j][m];
-            }
+            __syncthreads();   // sdt is restaged by the next chunk
         }
     } else {
-        if (has_head)
-            for (size_t i = lane; i < trf; i += 32) trec[i] = 0.f;
-        if (blockIdx.x == 0)
-            for (size_t i = threadIdx.x; i < (size_t)NP * CC; i += blockDim.x) grec[i] = 0.f;
-        if (threadIdx.x == 0 && T == 0) atomicOr(&p.err[b], RS_SEQ_ERR_EMPTY);
+        for (size_t i = threadIdx.x; i < (size_t)hpg * trf; i += blockDim.x) trec0[i] = 0.f;
+        for (int i = threadIdx.x; i < NP * CC; i += blockDim.x) grec[i] = 0.f;
+        if (T == 0 && g == 0 && threadIdx.x == 0) atomicOr(&p.err[b], RS_SEQ_ERR_EMPTY);
     }
 
     if (T > 0) {
-        // ---- append: the new entries into their ring slots
-        if (has_head) {
-            for (int t = 0; t < T; ++t) {
-                const int slot = (tail + t) & p.cap_mask;
-                copy_row(const_cast<unsigned char *>(xblk) + (size_t)slot * rowX, xraw + (size_t)(L_old + t) * rowX,
-                         (int)rowX, lane, 32);
-            }
-            for (int t = lane; t < T; t += 32)
-                const_cast<float *>(dtblk)[(tail + t) & p.cap_mask] = dt[L_old + t];
+        // ---- append: the new entries of the group's heads and the group's B, C rows
+        for (int t = 0; t < T; ++t) {
+            const int slot = (tail + t) & p.cap_mask;
+            copy_rows_cta(static_cast<unsigned char *>(p.ra) + ((size_t)b * H + h0) * p.blk_r + (size_t)slot * rowX,
+                          p.blk_r, static_cast<const unsigned char *>(in.x) + (((size_t)t * Bn + b) * H + h0) * rowX,
+                          hpg, (int)rowX);
         }
-        if (blockIdx.x == 0)
-            for (int t = warp; t < T; t += kPrepWarps) {
-                const int slot = (tail + t) & p.cap_mask;
-                copy_row(const_cast<unsigned char *>(bblk) + (size_t)slot * rowB,
-                         static_cast<const unsigned char *>(in.B) + (((size_t)t * Bn + b) * p.G + g) * rowB, (int)rowB, lane, 32);
-                copy_row(const_cast<unsigned char *>(cblk) + (size_t)slot * rowB,
-                         static_cast<const unsigned char *>(in.C) + (((size_t)t * Bn + b) * p.G + g) * rowB, (int)rowB, lane, 32);
-            }
-        arrive_and_advance(p, b, tail, T, gridDim.x * gridDim.y);
-        if (threadIdx.x == 0 && !ok) atomicOr(&p.err[b], RS_SEQ_ERR_EMPTY);
+        for (int w = threadIdx.x; w < hpg * T; w += blockDim.x) {
+            const int hl = w / T, t = w - (w / T) * T;
+            static_cast<float *>(p.rb)[((size_t)b * H + h0 + hl) * p.capd + ((tail + t) & p.cap_mask)] =
+                in.dt[((size_t)t * Bn + b) * H + h0 + hl];
+        }
+        for (int t = warp; t < T; t += kPrepWarps) {
+            const int slot = (tail + t) & p.cap_mask;
+            copy_row(bblk + (size_t)slot * rowB, b_row(L_old + t), (int)rowB, lane, 32);
+            copy_row(cblk + (size_t)slot * rowB, c_row(L_old + t), (int)rowB, lane, 32);
+        }
+        arrive_and_advance(p, b, tail, T, G);
     }
 }
 
 // -------------------------------------------------------------------- GDN --
 // One warp per (sequence, head); a CTA holds kPrepWarps heads of one sequence.
 // Per-warp shared memory (entries compact, buffer index i at row i):
-//   kraw [cap][CC] | vraw [cap][R] | qraw [NP][CC] | alpha [cap] | beta [cap] | coef [NP][cap]
+//   kraw [cap][CC] | qraw [NP][CC] | alpha [cap] | beta [cap]
 struct GdnPrepSmem {
-    size_t k, v, q, alpha, beta, coef, per_warp;
+    size_t k, q, alpha, beta, per_warp;
 };
 
-__host__ __device__ inline GdnPrepSmem gdn_prep_smem(int cap, int R, int CC, int NP, int ib) {
+__host__ __device__ inline GdnPrepSmem gdn_prep_smem(int cap, int CC, int NP, int ib) {
     GdnPrepSmem s;
     size_t w = 0;
     s.k = w;     w = align_up(w + (size_t)cap * CC * ib, 16);
-    s.v = w;     w = align_up(w + (size_t)cap * R * ib, 16);
     s.q = w;     w = align_up(w + (size_t)NP * CC * ib, 16);
     s.alpha = w; w = align_up(w + 4 * (size_t)cap, 16);
     s.beta = w;  w = align_up(w + 4 * (size_t)cap, 16);
-    s.coef = w;  w = align_up(w + 4 * (size_t)NP * cap, 16);
     s.per_warp = w;
     return s;
 }
@@ -304,37 +341,32 @@ __host__ __device__ inline GdnPrepSmem gdn_prep_smem(int cap, int R, int CC, int
 template <int CC, int NP>
 __global__ void __launch_bounds__(32 * kPrepWarps)
 gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
-    extern __shared__ __align__(16) unsigned char psm[];
-    __shared__ int s_head, s_tail;
+    extern __shared__ __align__(16) unsigned char psm_g[];
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int Bn = p.B, H = p.H, R = p.R, cap = p.cap, ib = p.in_dtype == RS_BF16 ? 2 : 4;
-    const int b = blockIdx.y;
-    const int h = blockIdx.x * kPrepWarps + warp;
+    const int cps = (H + kPrepWarps - 1) / kPrepWarps;   // CTAs per sequence
+    const int b = blockIdx.x / cps, hc = blockIdx.x - (blockIdx.x / cps) * cps;
+    const int h = hc * kPrepWarps + warp;
     const bool has_head = h < H;
-    const int tile = b * H + h;
-    const GdnPrepSmem S = gdn_prep_smem(cap, R, CC, NP, ib);
-    unsigned char *wsm = psm + (size_t)warp * S.per_warp;
-    unsigned char *kraw = wsm + S.k, *vraw = wsm + S.v, *qraw = wsm + S.q;
+    const size_t tile = (size_t)b * H + h;
+    const GdnPrepSmem S = gdn_prep_smem(cap, CC, NP, ib);
+    unsigned char *wsm = psm_g + (size_t)warp * S.per_warp;
+    unsigned char *kraw = wsm + S.k, *qraw = wsm + S.q;
     float *alpha = reinterpret_cast<float *>(wsm + S.alpha), *beta = reinterpret_cast<float *>(wsm + S.beta);
-    float *coef = reinterpret_cast<float *>(wsm + S.coef);
-    const size_t trf = tile_rec_floats(RS_GDN, NP, R, CC);
-    float *trec = p.rec + p.rec_tile_off + (size_t)tile * trf;
+    const size_t trf = tile_rec_floats(RS_GDN, NP, cap, CC);
+    float *trec = p.rec + p.rec_tile_off + tile * trf;
     const size_t rowC = (size_t)CC * ib, rowR = (size_t)R * ib;
 
-    if (threadIdx.x == 0) {
-        s_head = p.head[b];
-        s_tail = p.tail[b];
-    }
-    __syncthreads();
-    const int head = s_head, tail = s_tail, L_old = tail - head, L = L_old + T;
+    const int head = p.head[b], tail = p.tail[b];
+    const int L_old = tail - head, L = L_old + T;
     if (L_old < 0 || L > cap) {
         if (has_head)
             for (size_t i = lane; i < trf; i += 32) trec[i] = 0.f;
-        if (threadIdx.x == 0) atomicOr(&p.err[b], T > 0 ? RS_SEQ_ERR_OVERFLOW : RS_SEQ_ERR_EMPTY);
+        if (hc == 0 && threadIdx.x == 0) atomicOr(&p.err[b], T > 0 ? RS_SEQ_ERR_OVERFLOW : RS_SEQ_ERR_EMPTY);
         return;
     }
     const bool ok = npos >= 1 && L >= npos;
-    const size_t bh = has_head ? (size_t)tile : 0;
+    const size_t bh = has_head ? tile : 0;
     unsigned char *qblk = static_cast<unsigned char *>(p.ra) + bh * p.blk_c;
     unsigned char *kblk = static_cast<unsigned char *>(p.rb) + bh * p.blk_c;
     unsigned char *vblk = static_cast<unsigned char *>(p.rc) + bh * p.blk_r;
@@ -347,10 +379,7 @@ gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
     };
     if (has_head) {
         // ---- one round of asynchronous copies
-        for (int i = 0; i < L; ++i) {
-            stage_row(kraw + (size_t)i * rowC, src_row(kblk, in.k, rowC, i), (int)rowC, lane, 32);
-            if (ok) stage_row(vraw + (size_t)i * rowR, src_row(vblk, in.v, rowR, i), (int)rowR, lane, 32);
-        }
+        for (int i = 0; i < L; ++i) stage_row(kraw + (size_t)i * rowC, src_row(kblk, in.k, rowC, i), (int)rowC, lane, 32);
         if (ok)
             for (int j = 0; j < npos; ++j)
                 stage_row(qraw + (size_t)j * rowC, src_row(qblk, in.q, rowC, L - npos + j), (int)rowC, lane, 32);
@@ -363,7 +392,7 @@ gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
         __syncwarp();
 
         if (ok) {
-            float *mul = trec, *z = trec + 8, *vec = z + (size_t)NP * R;
+            float *coef = trec + kRecHdr, *vec = coef + (size_t)NP * cap;
             const float sc = p.gdn_scale;
             const float tscale = p.copy_dtype == RS_E4M3 ? p.scale[tile] : 1.f;
             constexpr int UPL = (CC + 31) / 32;
@@ -396,11 +425,14 @@ gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
                     if (j < npos) d[j] = warp_sum(d[j]);
 #pragma unroll
                 for (int j = 0; j < NP; ++j) {
-                    if (j < npos && i <= L - npos + j) {
+                    if (j >= npos) continue;
+                    if (i <= L - npos + j) {
                         const float f = bt * d[j];
-                        if (lane == 0) coef[j * cap + i] = f;
+                        if (lane == 0) coef[j * cap + i] = sc * f;
 #pragma unroll
                         for (int m = 0; m < UPL; ++m) u[j][m] = a * fmaf(-f, kr[m], u[j][m]);
+                    } else if (lane == 0) {
+                        coef[j * cap + i] = 0.f;
                     }
                 }
             }
@@ -412,37 +444,10 @@ gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
                         const int c = lane + 32 * m;
                         if (c < CC) vec[j * CC + c] = u[j][m];
                     }
-                    if (lane == 0) mul[j] = sc * tscale;
+                    if (lane == 0) trec[j] = sc * tscale;
                 }
             }
-            __syncwarp();
-            constexpr int RL = 8;   // rows per lane, R <= 256
-            float acc[NP][RL];
-#pragma unroll
-            for (int j = 0; j < NP; ++j)
-#pragma unroll
-                for (int m = 0; m < RL; ++m) acc[j][m] = 0.f;
-            for (int i = 0; i < L; ++i) {
-                float cf[NP];
-#pragma unroll
-                for (int j = 0; j < NP; ++j) cf[j] = (j < npos && i <= L - npos + j) ? coef[j * cap + i] : 0.f;
-#pragma unroll
-                for (int m = 0; m < RL; ++m) {
-                    const int r = lane + 32 * m;
-                    if (r >= R) break;
-                    const float vv = lds_in(vraw, (size_t)i * R + r, p.in_dtype);
-#pragma unroll
-                    for (int j = 0; j < NP; ++j) acc[j][m] = fmaf(cf[j], vv, acc[j][m]);
-                }
-            }
-#pragma unroll
-            for (int m = 0; m < RL; ++m) {
-                const int r = lane + 32 * m;
-                if (r >= R) break;
-#pragma unroll
-                for (int j = 0; j < NP; ++j)
-                    if (j < npos) z[j * R + r] = sc * acc[j][m];
-            }
+            if (lane == 0) write_header(trec, head, L, p.cap_mask);
         } else {
             for (size_t i = lane; i < trf; i += 32) trec[i] = 0.f;
         }
@@ -461,14 +466,14 @@ gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
             }
         }
     }
-    if (T > 0) arrive_and_advance(p, b, tail, T, gridDim.x);
-    if (threadIdx.x == 0 && !ok) atomicOr(&p.err[b], RS_SEQ_ERR_EMPTY);
+    if (T > 0) arrive_and_advance(p, b, tail, T, cps);
+    if (!ok && T == 0 && hc == 0 && threadIdx.x == 0) atomicOr(&p.err[b], RS_SEQ_ERR_EMPTY);
 }
 
 size_t prep_smem(const Params &p, int NP) {
     const int ib = p.in_dtype == RS_BF16 ? 2 : 4;
-    if (p.kind == RS_MAMBA2) return m2_prep_smem(p.cap, p.R, p.CC, NP, ib).total;
-    return kPrepWarps * gdn_prep_smem(p.cap, p.R, p.CC, NP, ib).per_warp;
+    if (p.kind == RS_MAMBA2) return 4 * m2_prep_floats(p.cap, NP, p.heads_per_group);
+    return kPrepWarps * gdn_prep_smem(p.cap, p.CC, NP, ib).per_warp;
 }
 
 template <int KIND, int CC, int NP>
@@ -478,14 +483,13 @@ static cudaError_t launch_prep_t(const Params &p, int npos, int T, const rs_inpu
         auto k = m2_prep_kernel<CC, NP>;
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        const dim3 grid((p.heads_per_group + kPrepWarps - 1) / kPrepWarps, p.G, p.B);
-        k<<<grid, 32 * kPrepWarps, smem, st>>>(p, npos, T, in);
+        k<<<(unsigned)((size_t)p.B * p.G), 32 * kPrepWarps, smem, st>>>(p, npos, T, in);
     } else {
         auto k = gdn_prep_kernel<CC, NP>;
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        const dim3 grid((p.H + kPrepWarps - 1) / kPrepWarps, p.B);
-        k<<<grid, 32 * kPrepWarps, smem, st>>>(p, npos, T, in);
+        const size_t cps = (p.H + kPrepWarps - 1) / kPrepWarps;
+        k<<<(unsigned)(cps * p.B), 32 * kPrepWarps, smem, st>>>(p, npos, T, in);
     }
     return cudaGetLastError();
 }
