@@ -23,7 +23,9 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-B, H, P, N, G, K_COMMIT, CAP, PREFILL = 256, 80, 64, 128, 1, 8, 16, 512
+B, H, P, N, G, K_COMMIT, CAP, PREFILL = 256, 80, 64, 128, 1, 8, 8, 512
+# Each decode step buffers one entry and every K_COMMIT-th step commits them
+# all, so the ring never holds more than K_COMMIT entries: CAP = K_COMMIT.
 POOL = 256          # distinct decode steps of inputs kept resident (cycled)
 METRIC = "SSM-layer decode tokens/s at batch 256; achieved HBM GB/s vs B200 peak"
 UNIT = "tokens/s"

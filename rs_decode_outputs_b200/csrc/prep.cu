@@ -80,6 +80,12 @@ __device__ __forceinline__ void arrive_and_advance(const Params &p, int b, int t
     }
 }
 
+// Let the streaming kernel queued behind this one start launching now (it
+// waits for this grid's results itself before it reads them).
+__device__ __forceinline__ void allow_dependent_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void write_header(float *trec, int head, int L, int cap_mask) {
     trec[kRecHeadSlot] = __int_as_float(head & cap_mask);
     trec[kRecLen] = __int_as_float(L);
@@ -104,14 +110,20 @@ __device__ __forceinline__ float chunk_dot(const uint4 &a, const uint4 &c, int i
 }
 
 // ---------------------------------------------------------------- Mamba-2 --
-// One CTA per (sequence, group).  Every global read is issued in bulk, with
-// no dependence between threads: the group's B_i . C_{e_j} are formed once
-// (lane groups of TPRB lanes per B row, the rows spread over the warps), and
-// dt of a chunk of up to kM2HeadChunk heads is staged for all entries at once;
-// then each warp takes heads of the chunk in turn (prefix sums of dt,
-// multipliers, coefficients) from shared memory, writing the head's record.
-// Shared memory: bc [NP][cap] | dt [HC][cap] | per warp: cum [cap].
-constexpr int kM2StageFloats = 4096;   // dt floats staged per round
+// One CTA per (sequence, group), built as a few rounds of independent global
+// reads with the arithmetic in between:
+//   1. reads that need no pointer: the first round of the new x rows (for the
+//      append) and A, D, the fp8 scales of the heads;
+//   2. the pointers;
+//   3. dt of every (head, entry), C_{e_j} and the B rows; the group's
+//      B_i . C_{e_j} (lane groups of TPRB lanes per B row, rows spread over the
+//      warps);
+//   4. per head (several heads per warp when L <= 16, one lane segment each):
+//      prefix sums of dt by segmented shuffles, multipliers, coefficients;
+//   5. the append stores and the tail.
+// Heads are taken in chunks of up to kM2HeadChunk per round of 3-4.
+// Shared memory: bc [NP][cap] | dt [HC][cap] | A, D, scale [HC] | per warp: cum [cap].
+constexpr int kM2StageFloats = 4096;   // dt floats staged per chunk
 
 __host__ __device__ inline int m2_head_chunk(int hpg, int cap) {
     const int hc = kM2StageFloats / cap;
@@ -119,60 +131,103 @@ __host__ __device__ inline int m2_head_chunk(int hpg, int cap) {
 }
 
 __host__ __device__ inline size_t m2_prep_floats(int cap, int NP, int hpg) {
-    return (size_t)NP * cap + (size_t)m2_head_chunk(hpg, cap) * cap + (size_t)kPrepWarps * cap;
+    const size_t hc = m2_head_chunk(hpg, cap);
+    return (size_t)NP * cap + hc * cap + 3 * hc + (size_t)kPrepWarps * cap;
 }
 
-// Copy `rows` rows of `row_bytes` bytes from a contiguous source to
-// dst0 + r * dst_stride with every thread of the CTA, loads issued ahead of
-// the stores; 16-, 4- or 2-byte units as the addresses allow.
-__device__ __forceinline__ void copy_rows_cta(unsigned char *dst0, size_t dst_stride, const unsigned char *src,
-                                              int rows, int row_bytes) {
-    const uintptr_t a = reinterpret_cast<uintptr_t>(dst0) | (uintptr_t)dst_stride |
-                        reinterpret_cast<uintptr_t>(src) | (uintptr_t)row_bytes;
-    const int unit = (a & 15) == 0 ? 16 : (a & 3) == 0 ? 4 : 2;
-    const int upr = row_bytes / unit, total = rows * upr;
-    constexpr int U = 4;
-    for (int k0 = threadIdx.x; k0 < total; k0 += U * blockDim.x) {
-        uint4 v[U];
+// A CTA-wide copy of `rows` rows of `row_bytes` bytes from a contiguous source
+// to dst0 + r * dst_stride, in 16-, 4- or 2-byte units as the addresses allow;
+// unit k of the copy is handled by thread k mod blockDim.
+struct RowCopy {
+    const unsigned char *src;
+    unsigned char *dst0;
+    size_t dst_stride;
+    int unit, upr, total;
+    static constexpr int U = 4;   // units a thread moves per round
+
+    __device__ void init(unsigned char *d0, size_t stride, const unsigned char *s, int rows, int row_bytes) {
+        const uintptr_t a = reinterpret_cast<uintptr_t>(d0) | (uintptr_t)stride |
+                            reinterpret_cast<uintptr_t>(s) | (uintptr_t)row_bytes;
+        src = s;
+        dst0 = d0;
+        dst_stride = stride;
+        unit = (a & 15) == 0 ? 16 : (a & 3) == 0 ? 4 : 2;
+        upr = row_bytes / unit;
+        total = rows * upr;
+    }
+    __device__ void load(uint4 (&v)[U], int k0) const {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int k = k0 + u * blockDim.x;
+            const int k = k0 + u * (int)blockDim.x;
             if (k >= total) break;
             const unsigned char *s = src + (size_t)k * unit;
             if (unit == 16) v[u] = *reinterpret_cast<const uint4 *>(s);
             else if (unit == 4) v[u].x = *reinterpret_cast<const uint32_t *>(s);
             else v[u].x = *reinterpret_cast<const uint16_t *>(s);
         }
+    }
+    __device__ void store(const uint4 (&v)[U], int k0, size_t dst_off) const {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int k = k0 + u * blockDim.x;
+            const int k = k0 + u * (int)blockDim.x;
             if (k >= total) break;
             const int r = k / upr, w = k - (k / upr) * upr;
-            unsigned char *d = dst0 + (size_t)r * dst_stride + (size_t)w * unit;
+            unsigned char *d = dst0 + dst_off + (size_t)r * dst_stride + (size_t)w * unit;
             if (unit == 16) *reinterpret_cast<uint4 *>(d) = v[u];
             else if (unit == 4) *reinterpret_cast<uint32_t *>(d) = v[u].x;
             else *reinterpret_cast<uint16_t *>(d) = static_cast<uint16_t>(v[u].x);
         }
     }
-}
+    // rounds from unit k_begin + threadIdx.x on: loads, then stores
+    __device__ void run(int k_begin, size_t dst_off) const {
+        for (int k0 = k_begin + threadIdx.x; k0 < total; k0 += U * blockDim.x) {
+            uint4 v[U];
+            load(v, k0);
+            store(v, k0, dst_off);
+        }
+    }
+};
 
 template <int CC, int NP>
 __global__ void __launch_bounds__(32 * kPrepWarps)
 m2_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
     extern __shared__ __align__(16) float psm[];
+    allow_dependent_launch();
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int Bn = p.B, H = p.H, R = p.R, cap = p.cap, G = p.G, hpg = p.heads_per_group;
     const int ib = p.in_dtype == RS_BF16 ? 2 : 4;
     const int b = blockIdx.x / G, g = blockIdx.x - (blockIdx.x / G) * G;
+    const int h0 = g * hpg;   // first head of the group
     const int HC = m2_head_chunk(hpg, cap);
     float *bc = psm;
-    float *sdt = psm + (size_t)NP * cap;
-    float *cum = sdt + (size_t)HC * cap + (size_t)warp * cap;
+    float *sdt = bc + (size_t)NP * cap;
+    float *sA = sdt + (size_t)HC * cap, *sD = sA + HC, *sS = sD + HC;
+    float *cum = sS + HC + (size_t)warp * cap;
     const size_t trf = tile_rec_floats(RS_MAMBA2, NP, cap, CC);
     float *grec = p.rec + ((size_t)b * G + g) * group_rec_floats(NP, CC);
-    float *trec0 = p.rec + p.rec_tile_off + ((size_t)b * H + (size_t)g * hpg) * trf;   // the group's heads
-    const int h0 = g * hpg;   // first head of the group
+    float *trec0 = p.rec + p.rec_tile_off + ((size_t)b * H + h0) * trf;   // the group's heads
+    const size_t rowB = (size_t)CC * ib, rowX = (size_t)R * ib;
+    const bool tscale_on = p.copy_dtype == RS_E4M3;
 
+    // ---- 1. reads that need no pointer
+    RowCopy xcopy;   // the new x rows of step 0 of the append, heads h0 .. h0 + hpg - 1
+    uint4 xfirst[RowCopy::U];
+    if (T > 0) {
+        xcopy.init(static_cast<unsigned char *>(p.ra) + ((size_t)b * H + h0) * p.blk_r, p.blk_r,
+                   static_cast<const unsigned char *>(in.x) + ((size_t)b * H + h0) * rowX, hpg, (int)rowX);
+        xcopy.load(xfirst, threadIdx.x);
+    }
+    auto stage_params = [&](int c0, int nh) {
+        for (int k = threadIdx.x; k < nh; k += blockDim.x) {
+            const int h = h0 + c0 + k;
+            sA[k] = p.A[h];
+            sD[k] = p.D ? p.D[h] : 0.f;
+            sS[k] = tscale_on ? p.scale[(size_t)b * H + h] : 1.f;
+        }
+    };
+    stage_params(0, hpg < HC ? hpg : HC);
+
+    // ---- 2. the pointers
     const int head = p.head[b], tail = p.tail[b];
     const int L_old = tail - head, L = L_old + T;
     if (L_old < 0 || L > cap) {   // corrupt pointers or ring overflow: nothing is appended
@@ -181,7 +236,6 @@ m2_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
         if (g == 0 && threadIdx.x == 0) atomicOr(&p.err[b], T > 0 ? RS_SEQ_ERR_OVERFLOW : RS_SEQ_ERR_EMPTY);
         return;
     }
-    const size_t rowB = (size_t)CC * ib, rowX = (size_t)R * ib;
     unsigned char *bblk = static_cast<unsigned char *>(p.rc) + ((size_t)b * G + g) * p.blk_c;
     unsigned char *cblk = static_cast<unsigned char *>(p.rd) + ((size_t)b * G + g) * p.blk_c;
     const float *dtring = static_cast<const float *>(p.rb) + ((size_t)b * H + h0) * p.capd;   // [hpg][capd]
@@ -198,10 +252,17 @@ m2_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
         return i < L_old ? dtring[(size_t)hl * p.capd + ((head + i) & p.cap_mask)]
                          : in.dt[((size_t)(i - L_old) * Bn + b) * H + h0 + hl];
     };
+    auto stage_dt = [&](int c0, int nh) {
+        for (int k = threadIdx.x; k < nh * L; k += blockDim.x) {
+            const int hl = k / L, i = k - (k / L) * L;
+            sdt[hl * cap + i] = dt_at(c0 + hl, i);
+        }
+    };
 
     const bool ok = npos >= 1 && L >= npos;
     if (ok) {
-        // ---- B_i . C_{e_j} for i < L (and the group record: C_{e_j} in fp32)
+        // ---- 3. dt, then B_i . C_{e_j} for i < L (and the group record: C_{e_j} in fp32)
+        stage_dt(0, hpg < HC ? hpg : HC);
         const int nch = CC * ib / 16;
         const int TPRB = nch < 32 ? nch : 32, CPLB = nch / TPRB, RPI = 32 / TPRB;
         const int q = lane % TPRB, sub = lane / TPRB;
@@ -214,7 +275,24 @@ m2_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
                 if (j < npos && c < CPLB)
                     cch[j][c] = reinterpret_cast<const uint4 *>(c_row(L - npos + j))[q + c * TPRB];
             }
-        if (warp == 0 && sub == 0) {
+        for (int i0 = warp * RPI; i0 < L; i0 += kPrepWarps * RPI) {
+            const int i = i0 + sub;
+            uint4 bch[2];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                bch[c] = make_uint4(0u, 0u, 0u, 0u);
+                if (i < L && c < CPLB) bch[c] = reinterpret_cast<const uint4 *>(b_row(i))[q + c * TPRB];
+            }
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+                if (j >= npos) break;
+                float d = chunk_dot(bch[0], cch[j][0], ib);
+                if (CPLB > 1) d += chunk_dot(bch[1], cch[j][1], ib);
+                for (int o = TPRB / 2; o >= 1; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+                if (q == 0 && i < L) bc[j * cap + i] = d;
+            }
+        }
+        if (warp == kPrepWarps - 1 && sub == 0) {
 #pragma unroll
             for (int j = 0; j < NP; ++j) {
                 if (j >= npos) break;
@@ -233,63 +311,71 @@ m2_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
                 }
             }
         }
-        for (int i0 = warp * RPI; i0 < L; i0 += kPrepWarps * RPI) {
-            const int i = i0 + sub;
-            uint4 bch[2];
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                bch[c] = make_uint4(0u, 0u, 0u, 0u);
-                if (i < L && c < CPLB) bch[c] = reinterpret_cast<const uint4 *>(b_row(i))[q + c * TPRB];
-            }
-#pragma unroll
-            for (int j = 0; j < NP; ++j) {
-                if (j >= npos) break;
-                float d = chunk_dot(bch[0], cch[j][0], ib);
-                if (CPLB > 1) d += chunk_dot(bch[1], cch[j][1], ib);
-                for (int o = TPRB / 2; o >= 1; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-                if (q == 0 && i < L) bc[j * cap + i] = d;
-            }
-        }
-        const bool tscale_on = p.copy_dtype == RS_E4M3;
+        __syncthreads();
+        // ---- 4. per head: prefix sums of dt, multipliers, coefficients
+        const int SW = L <= 1 ? 1 : L <= 2 ? 2 : L <= 4 ? 4 : L <= 8 ? 8 : L <= 16 ? 16 : 32;
         for (int c0 = 0; c0 < hpg; c0 += HC) {
             const int nh = hpg - c0 < HC ? hpg - c0 : HC;
-            // ---- dt of the chunk's heads, all entries at once
-            for (int k = threadIdx.x; k < nh * L; k += blockDim.x) {
-                const int hl = k / L, i = k - (k / L) * L;
-                sdt[hl * cap + i] = dt_at(c0 + hl, i);
+            if (c0 > 0) {   // next chunk of heads
+                __syncthreads();
+                stage_params(c0, nh);
+                stage_dt(c0, nh);
+                __syncthreads();
             }
-            __syncthreads();
-            // ---- per head: prefix sums of dt, multipliers, coefficients
-            for (int hc = warp; hc < nh; hc += kPrepWarps) {
-                const int hl = c0 + hc, h = h0 + hl;
-                const float *dts = sdt + (size_t)hc * cap;
-                float *trec = trec0 + (size_t)hl * trf;
-                float carry = 0.f;
-                for (int i0 = 0; i0 < L; i0 += 32) {
-                    const int i = i0 + lane;
-                    const float c = warp_incl_scan(i < L ? dts[i] : 0.f, lane) + carry;
-                    if (i < L) cum[i] = c;
-                    carry = __shfl_sync(0xffffffffu, c, 31);
-                }
-                __syncwarp();
-                const float A = p.A[h];
-                const float Dh = p.D ? p.D[h] : 0.f;
-                const float tscale = tscale_on ? p.scale[(size_t)b * H + h] : 1.f;
+            if (L <= 32) {
+                // lane segments of SW lanes, one head each, entry i = lane within the segment
+                const int nseg = 32 / SW, seg = lane / SW, i = lane - seg * SW;
+                for (int hb = warp * nseg; hb < nh; hb += kPrepWarps * nseg) {
+                    const int hc = hb + seg;
+                    const bool hv = hc < nh;
+                    const float dv = hv && i < L ? sdt[hc * cap + i] : 0.f;
+                    float c = dv;
+                    for (int o = 1; o < SW; o <<= 1) {
+                        const float t = __shfl_up_sync(0xffffffffu, c, o, SW);
+                        if (i >= o) c += t;
+                    }
+                    const float A = hv ? sA[hc] : 0.f, Dh = hv ? sD[hc] : 0.f, tsc = hv ? sS[hc] : 0.f;
+                    float *trec = trec0 + (size_t)(c0 + (hv ? hc : 0)) * trf;
 #pragma unroll
-                for (int j = 0; j < NP; ++j) {
-                    if (j >= npos) break;
-                    const int e = L - npos + j;
-                    const float ce = cum[e];
-                    if (lane == 0) trec[j] = expf(A * ce) * tscale;
-                    float *coef = trec + kRecHdr + (size_t)j * cap;
-                    for (int i = lane; i < L; i += 32)
-                        coef[i] = i <= e ? fmaf(expf(A * (ce - cum[i])) * dts[i], bc[j * cap + i], i == e ? Dh : 0.f)
-                                         : 0.f;
+                    for (int j = 0; j < NP; ++j) {
+                        if (j >= npos) break;
+                        const int e = L - npos + j;
+                        const float ce = __shfl_sync(0xffffffffu, c, e, SW);
+                        if (hv && i == 0) trec[j] = expf(A * ce) * tsc;
+                        if (hv && i < L)
+                            trec[kRecHdr + j * cap + i] =
+                                i <= e ? fmaf(expf(A * (ce - c)) * dv, bc[j * cap + i], i == e ? Dh : 0.f) : 0.f;
+                    }
+                    if (hv && i == 0) write_header(trec, head, L, p.cap_mask);
                 }
-                if (lane == 0) write_header(trec, head, L, p.cap_mask);
-                __syncwarp();   // cum is reused by the warp's next head
+            } else {
+                for (int hc = warp; hc < nh; hc += kPrepWarps) {
+                    const float *dts = sdt + (size_t)hc * cap;
+                    float *trec = trec0 + (size_t)(c0 + hc) * trf;
+                    float carry = 0.f;
+                    for (int i0 = 0; i0 < L; i0 += 32) {
+                        const int i = i0 + lane;
+                        const float c = warp_incl_scan(i < L ? dts[i] : 0.f, lane) + carry;
+                        if (i < L) cum[i] = c;
+                        carry = __shfl_sync(0xffffffffu, c, 31);
+                    }
+                    __syncwarp();
+                    const float A = sA[hc], Dh = sD[hc], tsc = sS[hc];
+#pragma unroll
+                    for (int j = 0; j < NP; ++j) {
+                        if (j >= npos) break;
+                        const int e = L - npos + j;
+                        const float ce = cum[e];
+                        if (lane == 0) trec[j] = expf(A * ce) * tsc;
+                        for (int i = lane; i < L; i += 32)
+                            trec[kRecHdr + j * cap + i] =
+                                i <= e ? fmaf(expf(A * (ce - cum[i])) * dts[i], bc[j * cap + i], i == e ? Dh : 0.f)
+                                       : 0.f;
+                    }
+                    if (lane == 0) write_header(trec, head, L, p.cap_mask);
+                    __syncwarp();   // cum is reused by the warp's next head
+                }
             }
-            __syncthreads();   // sdt is restaged by the next chunk
         }
     } else {
         for (size_t i = threadIdx.x; i < (size_t)hpg * trf; i += blockDim.x) trec0[i] = 0.f;
@@ -298,12 +384,14 @@ m2_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
     }
 
     if (T > 0) {
-        // ---- append: the new entries of the group's heads and the group's B, C rows
-        for (int t = 0; t < T; ++t) {
-            const int slot = (tail + t) & p.cap_mask;
-            copy_rows_cta(static_cast<unsigned char *>(p.ra) + ((size_t)b * H + h0) * p.blk_r + (size_t)slot * rowX,
-                          p.blk_r, static_cast<const unsigned char *>(in.x) + (((size_t)t * Bn + b) * H + h0) * rowX,
-                          hpg, (int)rowX);
+        // ---- 5. append: the new entries of the group's heads and the group's B, C rows
+        xcopy.store(xfirst, threadIdx.x, (size_t)(tail & p.cap_mask) * rowX);
+        xcopy.run(RowCopy::U * blockDim.x, (size_t)(tail & p.cap_mask) * rowX);   // units past the first round
+        for (int t = 1; t < T; ++t) {
+            RowCopy xc;
+            xc.init(static_cast<unsigned char *>(p.ra) + ((size_t)b * H + h0) * p.blk_r, p.blk_r,
+                    static_cast<const unsigned char *>(in.x) + (((size_t)t * Bn + b) * H + h0) * rowX, hpg, (int)rowX);
+            xc.run(0, (size_t)((tail + t) & p.cap_mask) * rowX);
         }
         for (int w = threadIdx.x; w < hpg * T; w += blockDim.x) {
             const int hl = w / T, t = w - (w / T) * T;
@@ -342,6 +430,7 @@ template <int CC, int NP>
 __global__ void __launch_bounds__(32 * kPrepWarps)
 gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
     extern __shared__ __align__(16) unsigned char psm_g[];
+    allow_dependent_launch();
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int Bn = p.B, H = p.H, R = p.R, cap = p.cap, ib = p.in_dtype == RS_BF16 ? 2 : 4;
     const int cps = (H + kPrepWarps - 1) / kPrepWarps;   // CTAs per sequence

@@ -85,6 +85,11 @@ __device__ __forceinline__ void bulk_pieces(void *dst, const void *src, uint32_t
     }
 }
 
+// Programmatic dependent launch: wait until the grid this one depends on (the
+// prep kernel before it in the stream) has completed and its writes are
+// visible; a no-op when the launch has no such dependency.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t policy_evict_last() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
@@ -102,7 +107,7 @@ __device__ __forceinline__ void load_vec_global(float (&v)[NP][CPT * VEC], const
 #pragma unroll
             for (int e = 0; e < VEC; e += 4) {
                 float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (j < npos) f = __ldg(reinterpret_cast<const float4 *>(vec + j * CC + (tl + c * TPR) * VEC + e));
+                if (j < npos) f = *reinterpret_cast<const float4 *>(vec + j * CC + (tl + c * TPR) * VEC + e);
                 v[j][c * VEC + e] = f.x;
                 v[j][c * VEC + e + 1] = f.y;
                 v[j][c * VEC + e + 2] = f.z;
@@ -153,11 +158,32 @@ stream_outputs_kernel(const Params p, const void *__restrict__ state, int npos, 
         if (lane == 0) {
             const uint64_t pol_state = policy_evict_first();
             const uint64_t pol_rec = policy_evict_last();
-            int team = 0, ms = 0, u = 0;   // team of stage k, its m % SPT and m / SPT
-            for (int k = 0; k < nst; ++k) {
+            // The checkpoint does not depend on the prep kernel that precedes
+            // this one in the stream, so the first ring's worth of checkpoint
+            // copies starts at once; the records and ring blocks the prep
+            // kernel writes are copied after griddepcontrol.wait (the prep
+            // grid has finished and its writes are visible).
+            const int pre = nst < S ? nst : S;
+            for (int k = 0; k < pre; ++k) {   // stage k < S: slot k % NT * SPT + k / NT, first use
+                const int s = (k % RL::NT) * SPT + k / RL::NT;
+                const int first = t0 + k * TT, cnt = nt - k * TT < TT ? nt - k * TT : TT;
+                mbar_expect_tx(full + s, cnt * (tile_bytes + blk_bytes + rec_bytes));
+                bulk_pieces(stage(s), static_cast<const unsigned char *>(state) + (size_t)first * tile_bytes,
+                            cnt * tile_bytes, full + s, pol_state);
+            }
+            grid_dependency_wait();
+            for (int k = 0; k < pre; ++k) {
+                const int s = (k % RL::NT) * SPT + k / RL::NT;
+                const int first = t0 + k * TT, cnt = nt - k * TT < TT ? nt - k * TT : TT;
+                unsigned char *st = stage(s);
+                bulk_pieces(st + lay.rec_off, trec + (size_t)first * rfl, cnt * rec_bytes, full + s, pol_rec);
+                bulk_pieces(st + lay.blk_off, wring + (size_t)first * blk_bytes, cnt * blk_bytes, full + s, pol_rec);
+            }
+            int team = 0, ms = 0, u = 1;   // stage S: team 0, m = SPT -> m % SPT = 0, m / SPT = 1
+            for (int k = pre; k < nst; ++k) {
                 const int s = team * SPT + ms;
                 const int first = t0 + k * TT, cnt = nt - k * TT < TT ? nt - k * TT : TT;
-                if (u >= 1 && !mbar_wait_bounded(empty + s, (u - 1) & 1)) {
+                if (!mbar_wait_bounded(empty + s, (u - 1) & 1)) {
                     atomicOr(&p.err[first / H], RS_SEQ_ERR_TIMEOUT);
                     break;
                 }
@@ -198,6 +224,7 @@ stream_outputs_kernel(const Params p, const void *__restrict__ state, int npos, 
     const int niter = (R + GROUPS * RG - 1) / (GROUPS * RG);
     float v[NP][CPT * VEC];
     int cur_bg = -1;   // (sequence, group) whose C vectors v holds (Mamba-2)
+    grid_dependency_wait();   // the group records are the prep kernel's output
     for (int m = 0; m * RL::NT + team < nst; ++m) {
         const int k = m * RL::NT + team, s = team * SPT + m % SPT, u = m / SPT;
         const int first = t0 + k * TT, cnt = nt - k * TT < TT ? nt - k * TT : TT;
@@ -364,8 +391,18 @@ static cudaError_t launch_stream_t(const Params &p, int npos, void *y, cudaStrea
     const int tiles = p.B * p.H;
     int grid = num_sms();
     if (grid > tiles) grid = tiles;
-    k<<<grid, Roles<NP>::THREADS, lay.total, st>>>(p, state, npos, y);
-    return cudaGetLastError();
+    // may start while the prep kernel before it is still running (see grid_dependency_wait)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(Roles<NP>::THREADS);
+    cfg.dynamicSmemBytes = lay.total;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, p, state, npos, y);
 }
 
 template <int KIND, int CC, typename TS>
