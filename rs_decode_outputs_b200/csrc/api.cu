@@ -7,6 +7,8 @@
 #include <new>
 #include <vector>
 
+#include <cuda.h>
+
 #include "launch.h"
 #include "outputs.cuh"
 #include "regtile.cuh"
@@ -129,6 +131,7 @@ bool has_inputs(int kind, int in_dtype, const rs_inputs *in) {
 }  // namespace
 
 struct rs_ctx {
+    alignas(64) unsigned char state_map[128];   // CUtensorMap of the checkpoint the outputs read
     rs_config cfg;
     rs_layout lay;
     rs::Params p;
@@ -241,6 +244,9 @@ rs_status rs_create(const rs_config *cfg, void *workspace, size_t workspace_byte
         delete h;
         return RS_ERR_UNSUPPORTED;
     }
+    static_assert(sizeof(CUtensorMap) == sizeof(h->state_map), "tensor map storage");
+    e = rs::make_state_map(p, h->state_map);
+    if (e != cudaSuccess) { delete h; return cuda_fail(e, "cuTensorMapEncodeTiled"); }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     e = cudaMemsetAsync(workspace, 0, L.total, st);
     if (e != cudaSuccess) { delete h; return cuda_fail(e, "cudaMemsetAsync"); }
@@ -314,7 +320,7 @@ rs_status rs_append(rs_handle h, const rs_inputs *in, int T, rs_stream stream) {
 static rs_status outputs(rs_handle h, int npos, void *y, rs_stream stream) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const rs_inputs none{};
-    return launched(rs::launch_outputs(h->p, npos, 0, none, y, st, prof_slot(h)), "outputs", 2);
+    return launched(rs::launch_outputs(h->p, h->state_map, npos, 0, none, y, st, prof_slot(h)), "outputs", 2);
 }
 
 rs_status rs_decode_outputs(rs_handle h, void *y, rs_stream stream) {
@@ -326,7 +332,7 @@ rs_status rs_decode_step(rs_handle h, const rs_inputs *in, int T, void *y, rs_st
     if (!h || !y || !has_inputs(h->cfg.kind, h->cfg.in_dtype, in)) return RS_ERR_ARG;
     if (T < 1) return RS_ERR_ARG;
     if (T > h->cfg.npos_max || T > h->cfg.cap) return RS_ERR_CAPACITY;
-    return launched(rs::launch_outputs(h->p, T, T, *in, y, static_cast<cudaStream_t>(stream), prof_slot(h)),
+    return launched(rs::launch_outputs(h->p, h->state_map, T, T, *in, y, static_cast<cudaStream_t>(stream), prof_slot(h)),
                     "decode_step", 2);
 }
 

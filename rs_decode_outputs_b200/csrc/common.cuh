@@ -111,11 +111,11 @@ __device__ __forceinline__ uint32_t pack_e4m3x2(float a, float b) {
 // A state tile is R rows of CC contiguous elements.  It is read in 16-byte
 // chunks; TPR threads share a row, each taking CPT chunks of it, strided by TPR
 // so that TPR neighbouring threads cover TPR * 16 contiguous bytes.
-template <int CC, int EB>
+template <int CC, int EB, int TPR_MAX = 8>
 struct Geom {
     static constexpr int VEC = 16 / EB;          // elements per chunk
     static constexpr int CHUNKS = CC / VEC;      // chunks per row
-    static constexpr int TPR = CHUNKS < 8 ? CHUNKS : 8;
+    static constexpr int TPR = CHUNKS < TPR_MAX ? CHUNKS : TPR_MAX;
     static constexpr int CPT = CHUNKS / TPR;     // chunks per thread per row
     static_assert(CC * EB >= 16, "row must hold at least one 16-byte chunk");
     static_assert(CHUNKS % TPR == 0, "chunks must split evenly");

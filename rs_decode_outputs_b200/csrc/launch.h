@@ -41,10 +41,14 @@ namespace rs {
 // record per tile into p.rec, then the streaming pass reads every checkpoint
 // tile once.  launch_outputs does both.
 cudaError_t launch_prep(const Params &p, int npos, int T, const rs_inputs &in, cudaStream_t st);
-// ev (may be NULL): three events recorded before the prep kernel, between the
-// two kernels and after the streaming kernel.
-cudaError_t launch_outputs(const Params &p, int npos, int T, const rs_inputs &in, void *y, cudaStream_t st,
-                           cudaEvent_t *ev = nullptr);
+// state_map: the CUtensorMap (host memory) of the checkpoint the outputs read,
+// from make_state_map.  ev (may be NULL): three events recorded before the
+// prep kernel, between the two kernels and after the streaming kernel.
+cudaError_t launch_outputs(const Params &p, const void *state_map, int npos, int T, const rs_inputs &in, void *y,
+                           cudaStream_t st, cudaEvent_t *ev = nullptr);
+// Encode the tensor map of the checkpoint the outputs read (the copy, or the
+// master without one) into map_out (a CUtensorMap, 64-byte aligned).
+cudaError_t make_state_map(const Params &p, void *map_out);
 size_t prep_smem(const Params &p, int NP);
 size_t stream_outputs_smem(const Params &p, int npos);
 

@@ -11,11 +11,14 @@
 //
 // The pass is bound by HBM bandwidth.  One CTA per SM runs over a contiguous
 // range of tiles with a shared-memory ring of stages.  A stage holds TT
-// consecutive tiles (about 32 KB, so that each bulk copy moves enough bytes
-// to keep the copy engine's per-operation cost small), their TT ring blocks
-// and their TT records: three 1-D bulk copies per stage, issued by one
-// producer thread in tile order (transaction-counted "full" barrier,
-// checkpoint evict-first in L2).  NT
+// consecutive tiles (about 32 KB, so that each copy moves enough bytes to keep
+// the copy engine's per-operation cost small), their TT ring blocks and their
+// TT records.  The tiles come in by 2-D tensor-map copies of boxes of up to 128
+// bytes of each row, swizzled in shared memory (16-byte chunk c of row r at
+// chunk c ^ (r mod 8) for 128-byte boxes) so that the tensor-core fragment
+// loads of the verification path are free of bank conflicts; the blocks and
+// records by 1-D bulk copies.  One producer thread issues them in tile order
+// (transaction-counted "full" barrier, checkpoint evict-first in L2).  NT
 // teams of four consumer warps take the stages in turn (stage k goes to team
 // k mod NT); each team owns SPT stages of the ring, which it uses in order,
 // and frees a stage ("empty" barrier) once it has contracted all its tiles.
@@ -23,10 +26,19 @@
 // same waiters, so a phase-parity wait never aliases an older phase.  Every
 // wait is bounded: one that gives up sets RS_SEQ_ERR_TIMEOUT and the role stops.
 //
+// Contraction.  One output position (decode) or an fp32 / fp8 copy: CUDA
+// cores, each lane group of TPR lanes owning RG rows at a time, fp32 FMAs.
+// Several positions over a bf16 copy (verification): bf16 tensor-core MMAs
+// (m16n8k16, fp32 accumulation) of 16-row blocks of the tile against the
+// position vectors, each vector split into a bf16 high part and a bf16
+// remainder (two MMAs per k-step), which keeps about 16 significant bits.
+//
 // Mamba-2's contraction vector C_{e_j} is one per (sequence, group) and is the
 // same for all heads of the group: the consumers keep it in registers and
-// reload it (plain cached loads, issued before the stage wait) only when the
-// group changes.
+// reload it only when the group changes.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "outputs.cuh"
 #include "launch.h"
 
@@ -37,6 +49,7 @@ constexpr int kTeamThreads = 32 * kTeamWarps;
 constexpr size_t kStreamSmemBudget = 224 * 1024;
 constexpr size_t kStageTarget = 32 * 1024;      // checkpoint bytes a stage aims for
 constexpr int kMaxTilesPerStage = 8;
+constexpr int kMaxBoxRows = 256;                // tensor-map box height limit
 
 template <int NP>
 struct Roles {
@@ -45,28 +58,47 @@ struct Roles {
     static constexpr int THREADS = 32 * (NCW + 1);    // + the producer warp
 };
 
+// Width of the boxes a checkpoint row is copied in, and the matching swizzle:
+// 16-byte chunk bits [4, 4 + log2(BOXB / 16)) of a shared-memory offset are
+// XORed with the bits from 7 up (the hardware's 32/64/128-byte swizzles).
+__host__ __device__ constexpr int box_bytes_for(int row_bytes) { return row_bytes < 128 ? row_bytes : 128; }
+__host__ __device__ constexpr uint32_t swizzle_mask_for(int box_bytes) {
+    return box_bytes == 128 ? 7u : box_bytes == 64 ? 3u : box_bytes == 32 ? 1u : 0u;
+}
+
+// Tiles per stage: about kStageTarget bytes, at most kMaxTilesPerStage, and
+// no more rows than one box may have.
+__host__ __device__ inline int stage_tiles(int R, size_t row_bytes) {
+    size_t tt = kStageTarget / ((size_t)R * row_bytes);
+    tt = tt < 1 ? 1 : tt > (size_t)kMaxTilesPerStage ? (size_t)kMaxTilesPerStage : tt;
+    const size_t by_rows = (size_t)kMaxBoxRows / (size_t)R;
+    return (int)(tt < by_rows ? tt : by_rows);
+}
+
 struct StreamLayout {
-    size_t blk_off, rec_off, stage_bytes, bars, total;
-    int TT;       // tiles per stage
-    int S, SPT;   // stages in all, stages per team
+    size_t box_region, blk_off, rec_off, stage_bytes, bars, total;
+    int TT;         // tiles per stage
+    int box_rows;   // rows of every box copy (TT R)
+    int S, SPT;     // stages in all, stages per team
 };
 
-// Stage: TT tiles (padded to 128 bytes) | TT ring blocks | TT tile records.
-__host__ __device__ inline StreamLayout stream_layout(size_t tile_bytes, size_t blk_bytes, size_t rec_bytes,
+// Stage (1024-byte aligned): nbox boxes of TT R rows | TT ring blocks | TT records.
+__host__ __device__ inline StreamLayout stream_layout(int R, size_t row_bytes, size_t blk_bytes, size_t rec_bytes,
                                                       int nt) {
     StreamLayout l;
-    size_t tt = kStageTarget / tile_bytes;
-    tt = tt < 1 ? 1 : tt > (size_t)kMaxTilesPerStage ? (size_t)kMaxTilesPerStage : tt;
-    l.TT = (int)tt;
-    l.blk_off = align_up(tt * tile_bytes, 128);
-    l.rec_off = align_up(l.blk_off + tt * blk_bytes, 16);
-    l.stage_bytes = align_up(l.rec_off + tt * rec_bytes, 128);
-    size_t spt = (kStreamSmemBudget - 1024) / (l.stage_bytes + 16) / nt;
+    l.TT = stage_tiles(R, row_bytes);
+    l.box_rows = l.TT * R;
+    const size_t boxb = (size_t)box_bytes_for((int)row_bytes), nbox = row_bytes / boxb;
+    l.box_region = align_up((size_t)l.box_rows * boxb, 1024);
+    l.blk_off = nbox * l.box_region;
+    l.rec_off = align_up(l.blk_off + (size_t)l.TT * blk_bytes, 16);
+    l.stage_bytes = align_up(l.rec_off + (size_t)l.TT * rec_bytes, 1024);
+    size_t spt = (kStreamSmemBudget - 2048) / (l.stage_bytes + 16) / nt;
     spt = spt < 1 ? 1 : spt > 8 ? 8 : spt;
     l.S = (int)(spt * nt);
     l.SPT = (int)spt;
     l.bars = (size_t)l.S * l.stage_bytes;
-    l.total = l.bars + align_up(16 * (size_t)l.S, 128);
+    l.total = l.bars + align_up(16 * (size_t)l.S, 128) + 1024;   // + slack to align the base to 1024
     return l;
 }
 
@@ -85,6 +117,16 @@ __device__ __forceinline__ void bulk_pieces(void *dst, const void *src, uint32_t
     }
 }
 
+// 2-D tensor-map copy of one box at element column x, row y (no multicast).
+__device__ __forceinline__ void tma_box_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar,
+                                           uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
 // Programmatic dependent launch: wait until the grid this one depends on (the
 // prep kernel before it in the stream) has completed and its writes are
 // visible; a no-op when the launch has no such dependency.
@@ -96,10 +138,33 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
     return p;
 }
 
-// The contraction vectors a consumer thread needs: vec_j at its CPT chunks.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&a)[4], const void *smem_row) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+                 : "r"(smem_u32(smem_row)));
+}
+
+// D += A B for one m16n8k16 bf16 tile with fp32 accumulation.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                 "{%8, %9}, {%0, %1, %2, %3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// bf16 pair (first value in the low half) rounded to nearest even, and the
+// pair of the remainders: hi + lo hold each fp32 value to about 16 bits.
+__device__ __forceinline__ void split_bf16x2(float v0, float v1, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat16 h0 = __float2bfloat16_rn(v0), h1 = __float2bfloat16_rn(v1);
+    const __nv_bfloat16 l0 = __float2bfloat16_rn(v0 - __bfloat162float(h0));
+    const __nv_bfloat16 l1 = __float2bfloat16_rn(v1 - __bfloat162float(h1));
+    hi = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+    lo = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+}
+
+// The contraction vectors a CUDA-core consumer thread needs: vec_j at its CPT chunks.
 template <int NP, int CPT, int VEC, int TPR>
-__device__ __forceinline__ void load_vec_global(float (&v)[NP][CPT * VEC], const float *__restrict__ vec,
-                                                int CC, int npos, int tl) {
+__device__ __forceinline__ void load_vec(float (&v)[NP][CPT * VEC], const float *vec, int CC, int npos, int tl) {
 #pragma unroll
     for (int j = 0; j < NP; ++j)
 #pragma unroll
@@ -115,22 +180,41 @@ __device__ __forceinline__ void load_vec_global(float (&v)[NP][CPT * VEC], const
             }
 }
 
+// The B fragments of the MMA path: vec_n (n = lane / 4 < npos, else 0) at
+// k = 16 ks + 2 (lane % 4) + {0, 1} and + 8, split into bf16 high and low parts.
+template <int KS>
+__device__ __forceinline__ void load_vec_frag(uint32_t (&bh)[KS][2], uint32_t (&bl)[KS][2], const float *vec,
+                                              int CC, int npos, int lane) {
+    const int n = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float2 f = make_float2(0.f, 0.f);
+            if (n < npos) f = *reinterpret_cast<const float2 *>(vec + n * CC + ks * 16 + 2 * t + 8 * h);
+            split_bf16x2(f.x, f.y, bh[ks][h], bl[ks][h]);
+        }
+}
+
 template <int KIND, int CC, typename TS, int NP>
 __global__ void __launch_bounds__(Roles<NP>::THREADS, 1)
-stream_outputs_kernel(const Params p, const void *__restrict__ state, int npos, void *y) {
+stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, int npos, void *y) {
     using RL = Roles<NP>;
-    extern __shared__ __align__(128) unsigned char smem[];
-    const int R = p.R, H = p.H;
-    const uint32_t tile_bytes = static_cast<uint32_t>(R) * CC * TS::bytes;
-    const int cap = p.cap;
+    constexpr int ROWB = CC * TS::bytes, BOXB = box_bytes_for(ROWB), NBOX = ROWB / BOXB, CPB = BOXB / 16;
+    constexpr uint32_t SWM = swizzle_mask_for(BOXB);
+    constexpr bool USE_MMA = TS::bytes == 2 && NP >= 2;   // bf16 copy, several positions
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const int R = p.R, H = p.H, cap = p.cap;
     const size_t rfl = tile_rec_floats(KIND, NP, cap, CC);
     const uint32_t rec_bytes = static_cast<uint32_t>(4 * rfl);
     const uint32_t blk_bytes = static_cast<uint32_t>(p.blk_r);
     const float *trec = p.rec + p.rec_tile_off;
     // ring rows the outputs sum over: Mamba-2 x, GDN v ([B][H][cap][R] blocks)
     const unsigned char *wring = static_cast<const unsigned char *>(KIND == RS_MAMBA2 ? p.ra : p.rc);
-    const StreamLayout lay = stream_layout(tile_bytes, blk_bytes, rec_bytes, RL::NT);
+    const StreamLayout lay = stream_layout(R, ROWB, blk_bytes, rec_bytes, RL::NT);
     const int S = lay.S, SPT = lay.SPT, TT = lay.TT;
+    const uint32_t stage_tx_tiles = static_cast<uint32_t>(NBOX * lay.box_rows * BOXB);
     // stage k of this CTA -> team k % NT, the team's m-th stage (m = k / NT),
     // ring slot (k % NT) * SPT + m % SPT, use m / SPT of that slot
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.bars);
@@ -158,6 +242,16 @@ stream_outputs_kernel(const Params p, const void *__restrict__ state, int npos, 
         if (lane == 0) {
             const uint64_t pol_state = policy_evict_first();
             const uint64_t pol_rec = policy_evict_last();
+            auto copy_tiles = [&](unsigned char *st, int first, uint64_t *bar) {
+                // a partial last stage still moves whole boxes (rows past the end read as zeros)
+#pragma unroll
+                for (int bx = 0; bx < NBOX; ++bx)
+                    tma_box_2d(st + bx * lay.box_region, &smap, bx * (BOXB / TS::bytes), first * R, bar, pol_state);
+            };
+            auto copy_side = [&](unsigned char *st, int first, int cnt, uint64_t *bar) {
+                bulk_pieces(st + lay.rec_off, trec + (size_t)first * rfl, cnt * rec_bytes, bar, pol_rec);
+                bulk_pieces(st + lay.blk_off, wring + (size_t)first * blk_bytes, cnt * blk_bytes, bar, pol_rec);
+            };
             // The checkpoint does not depend on the prep kernel that precedes
             // this one in the stream, so the first ring's worth of checkpoint
             // copies starts at once; the records and ring blocks the prep
@@ -167,17 +261,14 @@ stream_outputs_kernel(const Params p, const void *__restrict__ state, int npos, 
             for (int k = 0; k < pre; ++k) {   // stage k < S: slot k % NT * SPT + k / NT, first use
                 const int s = (k % RL::NT) * SPT + k / RL::NT;
                 const int first = t0 + k * TT, cnt = nt - k * TT < TT ? nt - k * TT : TT;
-                mbar_expect_tx(full + s, cnt * (tile_bytes + blk_bytes + rec_bytes));
-                bulk_pieces(stage(s), static_cast<const unsigned char *>(state) + (size_t)first * tile_bytes,
-                            cnt * tile_bytes, full + s, pol_state);
+                mbar_expect_tx(full + s, stage_tx_tiles + cnt * (blk_bytes + rec_bytes));
+                copy_tiles(stage(s), first, full + s);
             }
             grid_dependency_wait();
             for (int k = 0; k < pre; ++k) {
                 const int s = (k % RL::NT) * SPT + k / RL::NT;
                 const int first = t0 + k * TT, cnt = nt - k * TT < TT ? nt - k * TT : TT;
-                unsigned char *st = stage(s);
-                bulk_pieces(st + lay.rec_off, trec + (size_t)first * rfl, cnt * rec_bytes, full + s, pol_rec);
-                bulk_pieces(st + lay.blk_off, wring + (size_t)first * blk_bytes, cnt * blk_bytes, full + s, pol_rec);
+                copy_side(stage(s), first, cnt, full + s);
             }
             int team = 0, ms = 0, u = 1;   // stage S: team 0, m = SPT -> m % SPT = 0, m / SPT = 1
             for (int k = pre; k < nst; ++k) {
@@ -188,11 +279,9 @@ stream_outputs_kernel(const Params p, const void *__restrict__ state, int npos, 
                     break;
                 }
                 unsigned char *st = stage(s);
-                mbar_expect_tx(full + s, cnt * (tile_bytes + blk_bytes + rec_bytes));
-                bulk_pieces(st + lay.rec_off, trec + (size_t)first * rfl, cnt * rec_bytes, full + s, pol_rec);
-                bulk_pieces(st + lay.blk_off, wring + (size_t)first * blk_bytes, cnt * blk_bytes, full + s, pol_rec);
-                bulk_pieces(st, static_cast<const unsigned char *>(state) + (size_t)first * tile_bytes,
-                            cnt * tile_bytes, full + s, pol_state);
+                mbar_expect_tx(full + s, stage_tx_tiles + cnt * (blk_bytes + rec_bytes));
+                copy_side(st, first, cnt, full + s);
+                copy_tiles(st, first, full + s);
                 if (++team == RL::NT) {
                     team = 0;
                     if (++ms == SPT) {
@@ -207,154 +296,262 @@ stream_outputs_kernel(const Params p, const void *__restrict__ state, int npos, 
 
     // -------------------------------------------------------------- consumers
     // Team `team` (four warps) contracts stages team, team + NT, ...
-    using G = Geom<CC, TS::bytes>;
-    constexpr int VEC = G::VEC, TPR = G::TPR, CPT = G::CPT;
     const int team = warp / kTeamWarps;
-    const int ttid = threadIdx.x % kTeamThreads;
-    const int tl = ttid % TPR, row0 = ttid / TPR;
     const size_t y_pos_stride = (size_t)p.B * H * R;
     const int hpg = p.heads_per_group;
     const size_t gfl = group_rec_floats(NP, CC);
-    // A lane group (TPR lanes) covers RG rows per iteration: all RG x CPT chunks
-    // are loaded first, each row's partial dot goes to its own accumulator, and
-    // the RG partials are reduced across the group by a reduce-scatter, after
-    // which lane pair (2m, 2m+1) of the group holds the full sum of row m.
-    constexpr int RG = TPR == 8 ? 4 : 1;
-    constexpr int GROUPS = kTeamThreads / TPR;   // lane groups per team
-    const int niter = (R + GROUPS * RG - 1) / (GROUPS * RG);
-    float v[NP][CPT * VEC];
-    int cur_bg = -1;   // (sequence, group) whose C vectors v holds (Mamba-2)
+    // byte address of 16-byte chunk q of stage row rr (the swizzled box layout)
+    auto chunk_at = [&](const unsigned char *st, int rr, int q) -> const unsigned char * {
+        const int bx = q / CPB, c = q - bx * CPB;
+        const uint32_t o = static_cast<uint32_t>(rr) * BOXB + static_cast<uint32_t>(c) * 16u;
+        return st + (size_t)bx * lay.box_region + (o ^ (((o >> 7) & SWM) << 4));
+    };
     grid_dependency_wait();   // the group records are the prep kernel's output
-    for (int m = 0; m * RL::NT + team < nst; ++m) {
-        const int k = m * RL::NT + team, s = team * SPT + m % SPT, u = m / SPT;
-        const int first = t0 + k * TT, cnt = nt - k * TT < TT ? nt - k * TT : TT;
-        if (KIND == RS_MAMBA2) {   // issued before the wait, so the load overlaps it
-            const int b = first / H, bg = b * p.G + (first - b * H) / hpg;
-            if (bg != cur_bg) {
-                load_vec_global<NP, CPT, VEC, TPR>(v, p.rec + (size_t)bg * gfl, CC, npos, tl);
-                cur_bg = bg;
-            }
-        }
-        if (!mbar_wait_bounded(full + s, u & 1)) {
-            if (lane == 0) atomicOr(&p.err[first / H], RS_SEQ_ERR_TIMEOUT);
-            break;
-        }
-        const unsigned char *st = stage(s);
-        for (int i = 0; i < cnt; ++i) {
-            const int tile = first + i;
-            const unsigned char *tl_data = st + (size_t)i * tile_bytes;
-            const unsigned char *wblk = st + lay.blk_off + (size_t)i * blk_bytes;
-            const float *mul = reinterpret_cast<const float *>(st + lay.rec_off + (size_t)i * rec_bytes);
-            const int hs = __float_as_int(mul[kRecHeadSlot]);
-            const int Lr = min(max(__float_as_int(mul[kRecLen]), 0), cap);
-            const float *coef = mul + kRecHdr;
-            if (KIND == RS_MAMBA2) {
-                const int b = tile / H, bg = b * p.G + (tile - b * H) / hpg;
+
+    if constexpr (USE_MMA) {
+        // ----------------------------------------------- tensor-core path
+        constexpr int KS = CC / 16;
+        const int wt = warp % kTeamWarps;   // warp within the team
+        const int MB = (R + 15) / 16;       // 16-row blocks of a tile
+        uint32_t bh[KS][2], bl[KS][2];
+        int cur_bg = -1;
+        for (int m = 0; m * RL::NT + team < nst; ++m) {
+            const int k = m * RL::NT + team, s = team * SPT + m % SPT, u = m / SPT;
+            const int first = t0 + k * TT, cnt = nt - k * TT < TT ? nt - k * TT : TT;
+            if (KIND == RS_MAMBA2) {   // issued before the wait, so the loads overlap it
+                const int b = first / H, bg = b * p.G + (first - b * H) / hpg;
                 if (bg != cur_bg) {
-                    load_vec_global<NP, CPT, VEC, TPR>(v, p.rec + (size_t)bg * gfl, CC, npos, tl);
+                    load_vec_frag<KS>(bh, bl, p.rec + (size_t)bg * gfl, CC, npos, lane);
                     cur_bg = bg;
                 }
-            } else {
-                const float *vec = coef + (size_t)NP * cap;
-#pragma unroll
-                for (int j = 0; j < NP; ++j)
-#pragma unroll
-                    for (int c = 0; c < CPT; ++c)
-#pragma unroll
-                        for (int e = 0; e < VEC; ++e)
-                            v[j][c * VEC + e] = j < npos ? vec[j * CC + (tl + c * TPR) * VEC + e] : 0.f;
             }
-            float mj[NP];
-#pragma unroll
-            for (int j = 0; j < NP; ++j) mj[j] = j < npos ? mul[j] : 0.f;
-            const size_t y_off = (size_t)tile * R;
-            for (int it = 0; it < niter; ++it) {
-                const int rbase = (it * GROUPS + row0) * RG;   // first row of this group
-                uint4 raw[RG][CPT];
-#pragma unroll
-                for (int r = 0; r < RG; ++r)
-#pragma unroll
-                    for (int c = 0; c < CPT; ++c) {
-                        raw[r][c] = make_uint4(0u, 0u, 0u, 0u);
-                        if (rbase + r < R)
-                            raw[r][c] = *reinterpret_cast<const uint4 *>(
-                                tl_data + ((size_t)(rbase + r) * CC + (tl + c * TPR) * VEC) * TS::bytes);
-                    }
-                // even / odd columns accumulate in the two halves of packed fp32 FMAs
-                float2 acc2[NP][RG];
-#pragma unroll
-                for (int j = 0; j < NP; ++j)
-#pragma unroll
-                    for (int r = 0; r < RG; ++r) acc2[j][r] = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int r = 0; r < RG; ++r)
-#pragma unroll
-                    for (int c = 0; c < CPT; ++c) {
-                        float f[VEC];
-                        Chunk<TS>::expand(raw[r][c], f);
-#pragma unroll
-                        for (int e = 0; e < VEC; e += 2)
-#pragma unroll
-                            for (int j = 0; j < NP; ++j)
-                                acc2[j][r] = ffma2(make_float2(f[e], f[e + 1]),
-                                                   make_float2(v[j][c * VEC + e], v[j][c * VEC + e + 1]), acc2[j][r]);
-                    }
-                float acc[NP][RG];
-#pragma unroll
-                for (int j = 0; j < NP; ++j)
-#pragma unroll
-                    for (int r = 0; r < RG; ++r) acc[j][r] = acc2[j][r].x + acc2[j][r].y;
-                if constexpr (RG == 4) {
-                    const bool hi = tl & 4, b1 = tl & 2;
-                    const int row = rbase + (hi ? 2 : 0) + (b1 ? 1 : 0);
-                    // buffer terms of the row, entries split between the lane pair
-                    float zr[NP];
-#pragma unroll
-                    for (int j = 0; j < NP; ++j) zr[j] = 0.f;
-                    if (row < R)
-                        for (int e = tl & 1; e < Lr; e += 2) {
-                            const float w = lds_in(wblk, (size_t)((hs + e) & p.cap_mask) * R + row, p.in_dtype);
-#pragma unroll
-                            for (int j = 0; j < NP; ++j)
-                                if (j < npos) zr[j] = fmaf(coef[j * cap + e], w, zr[j]);
-                        }
-#pragma unroll
-                    for (int j = 0; j < NP; ++j) zr[j] += __shfl_xor_sync(0xffffffffu, zr[j], 1);
-#pragma unroll
-                    for (int j = 0; j < NP; ++j) {
-                        // xor 4: keep rows {0,1} (hi = 0) or {2,3} (hi = 1)
-                        const float k0 = (hi ? acc[j][2] : acc[j][0]) + __shfl_xor_sync(0xffffffffu, hi ? acc[j][0] : acc[j][2], 4);
-                        const float k1 = (hi ? acc[j][3] : acc[j][1]) + __shfl_xor_sync(0xffffffffu, hi ? acc[j][1] : acc[j][3], 4);
-                        // xor 2: keep the first (b1 = 0) or second (b1 = 1) of the pair
-                        float t = (b1 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, b1 ? k0 : k1, 2);
-                        t += __shfl_xor_sync(0xffffffffu, t, 1);
-                        if ((tl & 1) == 0 && row < R && j < npos)
-                            st_out(y, y_off + j * y_pos_stride + row, fmaf(mj[j], t, zr[j]), p.out_dtype);
+            if (!mbar_wait_bounded(full + s, u & 1)) {
+                if (lane == 0) atomicOr(&p.err[first / H], RS_SEQ_ERR_TIMEOUT);
+                break;
+            }
+            const unsigned char *st = stage(s);
+            for (int i = 0; i < cnt; ++i) {
+                const int tile = first + i;
+                const unsigned char *wblk = st + lay.blk_off + (size_t)i * blk_bytes;
+                const float *mul = reinterpret_cast<const float *>(st + lay.rec_off + (size_t)i * rec_bytes);
+                const int hs = __float_as_int(mul[kRecHeadSlot]);
+                const int Lr = min(max(__float_as_int(mul[kRecLen]), 0), cap);
+                const float *coef = mul + kRecHdr;
+                if (KIND == RS_MAMBA2) {
+                    const int b = tile / H, bg = b * p.G + (tile - b * H) / hpg;
+                    if (bg != cur_bg) {
+                        load_vec_frag<KS>(bh, bl, p.rec + (size_t)bg * gfl, CC, npos, lane);
+                        cur_bg = bg;
                     }
                 } else {
-                    // buffer terms of row rbase, entries split over the row's TPR lanes
-                    float zr[NP];
+                    load_vec_frag<KS>(bh, bl, coef + (size_t)NP * cap, CC, npos, lane);
+                }
+                const size_t y_off = (size_t)tile * R;
+                const int g = lane >> 2, t = lane & 3;
+                for (int mb = wt; mb < MB; mb += kTeamWarps) {
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+                    // ldmatrix rows: lane l addresses row (l & 7) + 8 ((l >> 3) & 1) of the block, chunk l >> 4
+                    int lr = mb * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                    lr = lr < R ? lr : R - 1;   // rows past the tile repeat its last row; their results are dropped
+                    const int rr = i * R + lr;
 #pragma unroll
-                    for (int j = 0; j < NP; ++j) zr[j] = 0.f;
-                    if (rbase < R)
-                        for (int e = tl; e < Lr; e += TPR) {
-                            const float w = lds_in(wblk, (size_t)((hs + e) & p.cap_mask) * R + rbase, p.in_dtype);
+                    for (int ks = 0; ks < KS; ++ks) {
+                        uint32_t a[4];
+                        ldmatrix_x4(a, chunk_at(st, rr, ks * 2 + (lane >> 4)));
+                        mma_bf16(d, a, bh[ks][0], bh[ks][1]);
+                        mma_bf16(d, a, bl[ks][0], bl[ks][1]);
+                    }
+                    // d[0], d[1]: row g, positions 2t, 2t + 1; d[2], d[3]: row g + 8
 #pragma unroll
-                            for (int j = 0; j < NP; ++j)
-                                if (j < npos) zr[j] = fmaf(coef[j * cap + e], w, zr[j]);
+                    for (int hr = 0; hr < 2; ++hr) {
+                        const int row = mb * 16 + g + 8 * hr;
+                        if (row >= R) continue;
+#pragma unroll
+                        for (int hc = 0; hc < 2; ++hc) {
+                            const int j = 2 * t + hc;
+                            if (j >= npos) continue;
+                            float z = 0.f;
+                            for (int e = 0; e < Lr; ++e)
+                                z = fmaf(coef[j * cap + e],
+                                         lds_in(wblk, (size_t)((hs + e) & p.cap_mask) * R + row, p.in_dtype), z);
+                            st_out(y, y_off + j * y_pos_stride + row, fmaf(mul[j], d[2 * hr + hc], z), p.out_dtype);
                         }
-#pragma unroll
-                    for (int j = 0; j < NP; ++j) {
-                        const float t = row_sum<TPR>(acc[j][0]);
-                        const float zz = row_sum<TPR>(zr[j]);
-                        if (tl == 0 && rbase < R && j < npos)
-                            st_out(y, y_off + j * y_pos_stride + rbase, fmaf(mj[j], t, zz), p.out_dtype);
                     }
                 }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + s);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty + s);
+    } else {
+        // ------------------------------------------------ CUDA-core path
+        // 8 lanes per row; 16 when many positions are contracted, so that each
+        // thread holds fewer columns of the NP vectors
+        using G = Geom<CC, TS::bytes, (NP >= 5 ? 16 : 8)>;
+        constexpr int VEC = G::VEC, TPR = G::TPR, CPT = G::CPT;
+        const int ttid = threadIdx.x % kTeamThreads;
+        const int tl = ttid % TPR, row0 = ttid / TPR;
+        // A lane group (TPR lanes) covers RG rows per iteration: all RG x CPT chunks
+        // are loaded first, each row's partial dot goes to its own accumulator, and
+        // the RG partials are reduced across the group by a reduce-scatter (TPR 8:
+        // lane pair (2m, 2m+1) of the group ends with row m; TPR 16: lanes 0-7 with
+        // row 0, lanes 8-15 with row 1).
+        constexpr int RG = TPR == 8 ? 4 : TPR == 16 ? 2 : 1;
+        constexpr int GROUPS = kTeamThreads / TPR;   // lane groups per team
+        const int niter = (R + GROUPS * RG - 1) / (GROUPS * RG);
+        float v[NP][CPT * VEC];
+        int cur_bg = -1;   // (sequence, group) whose C vectors v holds (Mamba-2)
+        for (int m = 0; m * RL::NT + team < nst; ++m) {
+            const int k = m * RL::NT + team, s = team * SPT + m % SPT, u = m / SPT;
+            const int first = t0 + k * TT, cnt = nt - k * TT < TT ? nt - k * TT : TT;
+            if (KIND == RS_MAMBA2) {   // issued before the wait, so the load overlaps it
+                const int b = first / H, bg = b * p.G + (first - b * H) / hpg;
+                if (bg != cur_bg) {
+                    load_vec<NP, CPT, VEC, TPR>(v, p.rec + (size_t)bg * gfl, CC, npos, tl);
+                    cur_bg = bg;
+                }
+            }
+            if (!mbar_wait_bounded(full + s, u & 1)) {
+                if (lane == 0) atomicOr(&p.err[first / H], RS_SEQ_ERR_TIMEOUT);
+                break;
+            }
+            const unsigned char *st = stage(s);
+            for (int i = 0; i < cnt; ++i) {
+                const int tile = first + i;
+                const unsigned char *wblk = st + lay.blk_off + (size_t)i * blk_bytes;
+                const float *mul = reinterpret_cast<const float *>(st + lay.rec_off + (size_t)i * rec_bytes);
+                const int hs = __float_as_int(mul[kRecHeadSlot]);
+                const int Lr = min(max(__float_as_int(mul[kRecLen]), 0), cap);
+                const float *coef = mul + kRecHdr;
+                if (KIND == RS_MAMBA2) {
+                    const int b = tile / H, bg = b * p.G + (tile - b * H) / hpg;
+                    if (bg != cur_bg) {
+                        load_vec<NP, CPT, VEC, TPR>(v, p.rec + (size_t)bg * gfl, CC, npos, tl);
+                        cur_bg = bg;
+                    }
+                } else {
+                    load_vec<NP, CPT, VEC, TPR>(v, coef + (size_t)NP * cap, CC, npos, tl);
+                }
+                float mj[NP];
+#pragma unroll
+                for (int j = 0; j < NP; ++j) mj[j] = j < npos ? mul[j] : 0.f;
+                const size_t y_off = (size_t)tile * R;
+                for (int it = 0; it < niter; ++it) {
+                    const int rbase = (it * GROUPS + row0) * RG;   // first row of this group
+                    uint4 raw[RG][CPT];
+#pragma unroll
+                    for (int r = 0; r < RG; ++r)
+#pragma unroll
+                        for (int c = 0; c < CPT; ++c) {
+                            raw[r][c] = make_uint4(0u, 0u, 0u, 0u);
+                            if (rbase + r < R)
+                                raw[r][c] = *reinterpret_cast<const uint4 *>(chunk_at(st, i * R + rbase + r, tl + c * TPR));
+                        }
+                    // even / odd columns accumulate in the two halves of packed fp32 FMAs
+                    float2 acc2[NP][RG];
+#pragma unroll
+                    for (int j = 0; j < NP; ++j)
+#pragma unroll
+                        for (int r = 0; r < RG; ++r) acc2[j][r] = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int r = 0; r < RG; ++r)
+#pragma unroll
+                        for (int c = 0; c < CPT; ++c) {
+                            float f[VEC];
+                            Chunk<TS>::expand(raw[r][c], f);
+#pragma unroll
+                            for (int e = 0; e < VEC; e += 2)
+#pragma unroll
+                                for (int j = 0; j < NP; ++j)
+                                    acc2[j][r] = ffma2(make_float2(f[e], f[e + 1]),
+                                                       make_float2(v[j][c * VEC + e], v[j][c * VEC + e + 1]), acc2[j][r]);
+                        }
+                    float acc[NP][RG];
+#pragma unroll
+                    for (int j = 0; j < NP; ++j)
+#pragma unroll
+                        for (int r = 0; r < RG; ++r) acc[j][r] = acc2[j][r].x + acc2[j][r].y;
+                    if constexpr (RG == 4) {
+                        const bool hi = tl & 4, b1 = tl & 2;
+                        const int row = rbase + (hi ? 2 : 0) + (b1 ? 1 : 0);
+                        // buffer terms of the row, entries split between the lane pair
+                        float zr[NP];
+#pragma unroll
+                        for (int j = 0; j < NP; ++j) zr[j] = 0.f;
+                        if (row < R)
+                            for (int e = tl & 1; e < Lr; e += 2) {
+                                const float w = lds_in(wblk, (size_t)((hs + e) & p.cap_mask) * R + row, p.in_dtype);
+#pragma unroll
+                                for (int j = 0; j < NP; ++j)
+                                    if (j < npos) zr[j] = fmaf(coef[j * cap + e], w, zr[j]);
+                            }
+#pragma unroll
+                        for (int j = 0; j < NP; ++j) zr[j] += __shfl_xor_sync(0xffffffffu, zr[j], 1);
+#pragma unroll
+                        for (int j = 0; j < NP; ++j) {
+                            // xor 4: keep rows {0,1} (hi = 0) or {2,3} (hi = 1)
+                            const float k0 = (hi ? acc[j][2] : acc[j][0]) + __shfl_xor_sync(0xffffffffu, hi ? acc[j][0] : acc[j][2], 4);
+                            const float k1 = (hi ? acc[j][3] : acc[j][1]) + __shfl_xor_sync(0xffffffffu, hi ? acc[j][1] : acc[j][3], 4);
+                            // xor 2: keep the first (b1 = 0) or second (b1 = 1) of the pair
+                            float t = (b1 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, b1 ? k0 : k1, 2);
+                            t += __shfl_xor_sync(0xffffffffu, t, 1);
+                            if ((tl & 1) == 0 && row < R && j < npos)
+                                st_out(y, y_off + j * y_pos_stride + row, fmaf(mj[j], t, zr[j]), p.out_dtype);
+                        }
+                    } else if constexpr (RG == 2) {
+                        // buffer terms of both rows, entries split over the group's 16 lanes
+                        float zr[2][NP];
+#pragma unroll
+                        for (int r = 0; r < 2; ++r)
+#pragma unroll
+                            for (int j = 0; j < NP; ++j) zr[r][j] = 0.f;
+                        for (int e = tl; e < Lr; e += TPR) {
+                            const size_t wrow = (size_t)((hs + e) & p.cap_mask) * R;
+#pragma unroll
+                            for (int r = 0; r < 2; ++r) {
+                                const float w = rbase + r < R ? lds_in(wblk, wrow + rbase + r, p.in_dtype) : 0.f;
+#pragma unroll
+                                for (int j = 0; j < NP; ++j)
+                                    if (j < npos) zr[r][j] = fmaf(coef[j * cap + e], w, zr[r][j]);
+                            }
+                        }
+                        const bool hi = tl & 8;
+                        const int row = rbase + (hi ? 1 : 0);
+#pragma unroll
+                        for (int j = 0; j < NP; ++j) {
+                            // each lane's share of both rows' outputs, then xor 8 keeps row 0 (hi = 0) or row 1
+                            const float o0 = fmaf(mj[j], acc[j][0], zr[0][j]), o1 = fmaf(mj[j], acc[j][1], zr[1][j]);
+                            float t = (hi ? o1 : o0) + __shfl_xor_sync(0xffffffffu, hi ? o0 : o1, 8);
+                            t += __shfl_xor_sync(0xffffffffu, t, 4);
+                            t += __shfl_xor_sync(0xffffffffu, t, 2);
+                            t += __shfl_xor_sync(0xffffffffu, t, 1);
+                            if ((tl & 7) == 0 && row < R && j < npos)
+                                st_out(y, y_off + j * y_pos_stride + row, t, p.out_dtype);
+                        }
+                    } else {
+                        // buffer terms of row rbase, entries split over the row's TPR lanes
+                        float zr[NP];
+#pragma unroll
+                        for (int j = 0; j < NP; ++j) zr[j] = 0.f;
+                        if (rbase < R)
+                            for (int e = tl; e < Lr; e += TPR) {
+                                const float w = lds_in(wblk, (size_t)((hs + e) & p.cap_mask) * R + rbase, p.in_dtype);
+#pragma unroll
+                                for (int j = 0; j < NP; ++j)
+                                    if (j < npos) zr[j] = fmaf(coef[j * cap + e], w, zr[j]);
+                            }
+#pragma unroll
+                        for (int j = 0; j < NP; ++j) {
+                            const float t = row_sum<TPR>(acc[j][0]);
+                            const float zz = row_sum<TPR>(zr[j]);
+                            if (tl == 0 && rbase < R && j < npos)
+                                st_out(y, y_off + j * y_pos_stride + rbase, fmaf(mj[j], t, zz), p.out_dtype);
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + s);
+        }
     }
 }
 
@@ -372,18 +569,49 @@ static int num_sms() {
     return g_num_sms[dev];
 }
 
+static int state_bytes(const Params &p) { return p.copy_dtype == RS_BF16 ? 2 : p.copy_dtype == RS_E4M3 ? 1 : 4; }
+
 static StreamLayout layout_for(const Params &p, int npos) {
-    const int eb = p.copy_dtype == RS_BF16 ? 2 : p.copy_dtype == RS_E4M3 ? 1 : 4;
     const int NPr = prep_np(npos);
     const int nt = NPr <= 2 ? Roles<1>::NT : Roles<8>::NT;
-    return stream_layout((size_t)p.R * p.CC * eb, p.blk_r, 4 * tile_rec_floats(p.kind, NPr, p.cap, p.CC), nt);
+    return stream_layout(p.R, (size_t)p.CC * state_bytes(p), p.blk_r, 4 * tile_rec_floats(p.kind, NPr, p.cap, p.CC), nt);
 }
 
 size_t stream_outputs_smem(const Params &p, int npos) { return layout_for(p, npos).total; }
 
+cudaError_t make_state_map(const Params &p, void *map_out) {
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (!encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return e;
+        if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    const int eb = state_bytes(p);
+    const size_t row_bytes = (size_t)p.CC * eb;
+    const int boxb = box_bytes_for((int)row_bytes);
+    void *base = p.copy_dtype == RS_NONE ? static_cast<void *>(p.master) : p.copy;
+    const CUtensorMapDataType dt = eb == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                   : eb == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                             : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const cuuint64_t dims[2] = {(cuuint64_t)p.CC, (cuuint64_t)p.B * p.H * p.R};
+    const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    const cuuint32_t box[2] = {(cuuint32_t)(boxb / eb), (cuuint32_t)(stage_tiles(p.R, row_bytes) * p.R)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapSwizzle swz = boxb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                   : boxb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                   : boxb == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                : CU_TENSOR_MAP_SWIZZLE_NONE;
+    const CUresult r = encode(static_cast<CUtensorMap *>(map_out), dt, 2, base, dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int KIND, int CC, typename TS, int NP>
-static cudaError_t launch_stream_t(const Params &p, int npos, void *y, cudaStream_t st) {
-    const void *state = p.copy_dtype == RS_NONE ? static_cast<const void *>(p.master) : p.copy;
+static cudaError_t launch_stream_t(const Params &p, const CUtensorMap &smap, int npos, void *y, cudaStream_t st) {
     const StreamLayout lay = layout_for(p, npos);
     auto k = stream_outputs_kernel<KIND, CC, TS, NP>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total);
@@ -402,36 +630,37 @@ static cudaError_t launch_stream_t(const Params &p, int npos, void *y, cudaStrea
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k, p, state, npos, y);
+    return cudaLaunchKernelEx(&cfg, k, p, smap, npos, y);
 }
 
 template <int KIND, int CC, typename TS>
-static cudaError_t launch_stream_np(const Params &p, int npos, void *y, cudaStream_t st) {
+static cudaError_t launch_stream_np(const Params &p, const CUtensorMap &smap, int npos, void *y, cudaStream_t st) {
     switch (prep_np(npos)) {
-        case 1: return launch_stream_t<KIND, CC, TS, 1>(p, npos, y, st);
-        case 2: return launch_stream_t<KIND, CC, TS, 2>(p, npos, y, st);
-        case 5: return launch_stream_t<KIND, CC, TS, 5>(p, npos, y, st);
-        default: return launch_stream_t<KIND, CC, TS, 8>(p, npos, y, st);
+        case 1: return launch_stream_t<KIND, CC, TS, 1>(p, smap, npos, y, st);
+        case 2: return launch_stream_t<KIND, CC, TS, 2>(p, smap, npos, y, st);
+        case 5: return launch_stream_t<KIND, CC, TS, 5>(p, smap, npos, y, st);
+        default: return launch_stream_t<KIND, CC, TS, 8>(p, smap, npos, y, st);
     }
 }
 
 template <int KIND>
 struct StreamCC {
     template <int CC>
-    static cudaError_t go(const Params &p, int npos, void *y, cudaStream_t st) {
+    static cudaError_t go(const Params &p, const CUtensorMap &smap, int npos, void *y, cudaStream_t st) {
         switch (p.copy_dtype) {
-            case RS_BF16: return launch_stream_np<KIND, CC, StBF16>(p, npos, y, st);
-            case RS_E4M3: return launch_stream_np<KIND, CC, StE4M3>(p, npos, y, st);
-            default: return launch_stream_np<KIND, CC, StF32>(p, npos, y, st);
+            case RS_BF16: return launch_stream_np<KIND, CC, StBF16>(p, smap, npos, y, st);
+            case RS_E4M3: return launch_stream_np<KIND, CC, StE4M3>(p, smap, npos, y, st);
+            default: return launch_stream_np<KIND, CC, StF32>(p, smap, npos, y, st);
         }
     }
 };
 
 // Output-only replay / verification, optionally preceded by the append of T
-// step inputs: the prep kernel (which also performs the append) writes the
-// records, then the streaming pass reads each checkpoint tile once.
-cudaError_t launch_outputs(const Params &p, int npos, int T, const rs_inputs &in, void *y, cudaStream_t st,
-                           cudaEvent_t *ev) {
+// step inputs: the prep kernel writes the per-tile records (and appends), then
+// the streaming pass reads each checkpoint tile once.
+cudaError_t launch_outputs(const Params &p, const void *state_map, int npos, int T, const rs_inputs &in, void *y,
+                           cudaStream_t st, cudaEvent_t *ev) {
+    const CUtensorMap &smap = *static_cast<const CUtensorMap *>(state_map);
     cudaError_t e;
     if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess) return e;
     e = launch_prep(p, npos, T, in, st);
@@ -439,9 +668,9 @@ cudaError_t launch_outputs(const Params &p, int npos, int T, const rs_inputs &in
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
     e = cudaErrorInvalidValue;
     if (p.kind == RS_MAMBA2) {
-        RS_DISPATCH_CC(p.CC, e = StreamCC<RS_MAMBA2>::go, (p, npos, y, st));
+        RS_DISPATCH_CC(p.CC, e = StreamCC<RS_MAMBA2>::go, (p, smap, npos, y, st));
     } else {
-        RS_DISPATCH_CC(p.CC, e = StreamCC<RS_GDN>::go, (p, npos, y, st));
+        RS_DISPATCH_CC(p.CC, e = StreamCC<RS_GDN>::go, (p, smap, npos, y, st));
     }
     if (e != cudaSuccess) return e;
     if (ev) e = cudaEventRecord(ev[2], st);

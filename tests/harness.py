@@ -1,12 +1,15 @@
 """Helpers shared by the GPU parity tests: run a workload through the CUDA
 library and the same inputs through the fp64 oracle, then compare.
 
-Error metric (the pages fix none): the normwise relative error of every
-(sequence, head) output vector, ||y_gpu - y_oracle||_2 / ||y_oracle||_2 over its
-R elements; a test reports the maximum over vectors and steps.  The same ratio
-in the infinity norm (rel_err_inf) is reported as a diagnostic: with an fp8
-copy its worst row can exceed the E4M3 unit roundoff through cancellation in
-the row's dot product, which the 2-norm averages over the vector.
+Error measure of the tolerances (the pages give "max relative error" and no
+norm): for each (sequence, head) output vector of R elements,
+||y_gpu - y_oracle||_inf / ||y_oracle||_inf, maximised over vectors and steps
+(rel_err).  The E4M3 copy is checked on a whole step's outputs in the same
+norm (rel_err_step): its 3 mantissa bits alone can move a single vector by
+more than the 6e-2 tolerance, whatever the kernels do, while the step-level
+ratio stays near the format's unit roundoff.  The low-precision kernels'
+own arithmetic is checked per vector against the oracle fed the same
+quantised checkpoint (QuantCheckpoint).
 """
 import numpy as np
 import torch
@@ -28,6 +31,17 @@ def f64(t):
 
 
 def rel_err(y, ref):
+    """The tolerances' error measure: max over the leading dims (sequence, head,
+    position) of ||y - ref||_inf / ||ref||_inf along the last axis, i.e. each
+    (sequence, head)'s output vector on its own."""
+    y = np.asarray(y, np.float64)
+    ref = np.asarray(ref, np.float64)
+    num = np.max(np.abs(y - ref), axis=-1)
+    den = np.maximum(np.max(np.abs(ref), axis=-1), 1e-300)
+    return float(np.max(num / den))
+
+
+def rel_err_2(y, ref):
     """max over leading dims of ||y - ref||_2 / ||ref||_2 along the last axis."""
     y = np.asarray(y, np.float64)
     ref = np.asarray(ref, np.float64)
@@ -36,29 +50,20 @@ def rel_err(y, ref):
     return float(np.max(num / den))
 
 
-def rel_err_inf(y, ref):
-    """max over leading dims of ||y - ref||_inf / ||ref||_inf along the last axis."""
+def rel_err_step(y, ref):
+    """||y - ref||_inf / ||ref||_inf over a whole step's outputs (all sequences,
+    heads and positions together)."""
     y = np.asarray(y, np.float64)
     ref = np.asarray(ref, np.float64)
-    num = np.max(np.abs(y - ref), axis=-1)
-    den = np.maximum(np.max(np.abs(ref), axis=-1), 1e-300)
-    return float(np.max(num / den))
-
-
-def rel_err_fro(y, ref):
-    """||y - ref||_F / ||ref||_F over the whole array (one step's outputs)."""
-    y = np.asarray(y, np.float64)
-    ref = np.asarray(ref, np.float64)
-    return float(np.sqrt(np.sum((y - ref) ** 2)) / max(np.sqrt(np.sum(ref ** 2)), 1e-300))
+    return float(np.max(np.abs(y - ref)) / max(np.max(np.abs(ref)), 1e-300))
 
 
 def out_err(y, ref, copy_dtype):
-    """The error measure each output-copy tolerance is read on: the largest
-    per-(sequence, head) relative 2-norm error for fp32 and bf16 checkpoints;
-    for the E4M3 copy (3 mantissa bits, so single output vectors of a tile can
-    lose more than the tolerance to rounding alone) the step's whole output in
-    the Frobenius norm."""
-    return rel_err_fro(y, ref) if copy_dtype == rs.RS_E4M3 else rel_err(y, ref)
+    """The measure each output-copy tolerance is checked on: per (sequence,
+    head) (rel_err) for fp32 and bf16 checkpoints; for the E4M3 copy, whose 3
+    mantissa bits alone can cost a single output vector more than the
+    tolerance, the step's whole output (rel_err_step)."""
+    return rel_err_step(y, ref) if copy_dtype == rs.RS_E4M3 else rel_err(y, ref)
 
 
 def torch_dtype(code):
