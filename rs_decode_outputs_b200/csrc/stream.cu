@@ -26,12 +26,15 @@
 // same waiters, so a phase-parity wait never aliases an older phase.  Every
 // wait is bounded: one that gives up sets RS_SEQ_ERR_TIMEOUT and the role stops.
 //
-// Contraction.  One output position (decode) or an fp32 / fp8 copy: CUDA
-// cores, each lane group of TPR lanes owning RG rows at a time, fp32 FMAs.
-// Several positions over a bf16 copy (verification): bf16 tensor-core MMAs
-// (m16n8k16, fp32 accumulation) of 16-row blocks of the tile against the
-// position vectors, each vector split into a bf16 high part and a bf16
-// remainder (two MMAs per k-step), which keeps about 16 significant bits.
+// Contraction.  Several positions over a bf16 copy (verification): bf16
+// tensor-core MMAs (m16n8k16, fp32 accumulation) of 16-row blocks of the tile
+// against the position vectors (up to 8 columns), each vector split into a
+// bf16 high part and a bf16 remainder (two MMAs per k-step), which keeps
+// about 16 significant bits; per element this costs far fewer instructions
+// than unpacking and FMAs.  One position (decode), or an fp32 / fp8 copy:
+// CUDA cores, each lane group of TPR lanes owning RG rows at a time, fp32
+// FMAs (for one position the MMA's 8 columns would be 7/8 idle, and the
+// measured CUDA-core pass is faster).
 //
 // Mamba-2's contraction vector C_{e_j} is one per (sequence, group) and is the
 // same for all heads of the group: the consumers keep it in registers and
@@ -46,7 +49,8 @@ namespace rs {
 
 constexpr int kTeamWarps = 4;                   // consumer warps per team (one tile at a time)
 constexpr int kTeamThreads = 32 * kTeamWarps;
-constexpr size_t kStreamSmemBudget = 224 * 1024;
+constexpr size_t kStreamSmemMax = 227 * 1024;     // opt-in shared memory of one CTA
+constexpr size_t kStreamSmemReserve = 1024 + 512; // base alignment slack + barriers
 constexpr size_t kStageTarget = 32 * 1024;      // checkpoint bytes a stage aims for
 constexpr int kMaxTilesPerStage = 8;
 constexpr int kMaxBoxRows = 256;                // tensor-map box height limit
@@ -93,7 +97,7 @@ __host__ __device__ inline StreamLayout stream_layout(int R, size_t row_bytes, s
     l.blk_off = nbox * l.box_region;
     l.rec_off = align_up(l.blk_off + (size_t)l.TT * blk_bytes, 16);
     l.stage_bytes = align_up(l.rec_off + (size_t)l.TT * rec_bytes, 1024);
-    size_t spt = (kStreamSmemBudget - 2048) / (l.stage_bytes + 16) / nt;
+    size_t spt = (kStreamSmemMax - kStreamSmemReserve) / l.stage_bytes / nt;
     spt = spt < 1 ? 1 : spt > 8 ? 8 : spt;
     l.S = (int)(spt * nt);
     l.SPT = (int)spt;
@@ -202,7 +206,7 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
     using RL = Roles<NP>;
     constexpr int ROWB = CC * TS::bytes, BOXB = box_bytes_for(ROWB), NBOX = ROWB / BOXB, CPB = BOXB / 16;
     constexpr uint32_t SWM = swizzle_mask_for(BOXB);
-    constexpr bool USE_MMA = TS::bytes == 2 && NP >= 2;   // bf16 copy, several positions
+    constexpr bool USE_MMA = TS::bytes == 2 && NP >= 2;   // bf16 copy, several positions: tensor cores
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int R = p.R, H = p.H, cap = p.cap;
@@ -318,8 +322,14 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
         for (int m = 0; m * RL::NT + team < nst; ++m) {
             const int k = m * RL::NT + team, s = team * SPT + m % SPT, u = m / SPT;
             const int first = t0 + k * TT, cnt = nt - k * TT < TT ? nt - k * TT : TT;
+            // (sequence, group) of the stage's first tile and its head within the
+            // group; consecutive tiles advance the head, and the group index
+            // b G + g by one whenever the head wraps
+            int bg = 0, hl = 0;
             if (KIND == RS_MAMBA2) {   // issued before the wait, so the loads overlap it
-                const int b = first / H, bg = b * p.G + (first - b * H) / hpg;
+                const int b = first / H, h = first - b * H, g = h / hpg;
+                bg = b * p.G + g;
+                hl = h - g * hpg;
                 if (bg != cur_bg) {
                     load_vec_frag<KS>(bh, bl, p.rec + (size_t)bg * gfl, CC, npos, lane);
                     cur_bg = bg;
@@ -338,7 +348,10 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
                 const int Lr = min(max(__float_as_int(mul[kRecLen]), 0), cap);
                 const float *coef = mul + kRecHdr;
                 if (KIND == RS_MAMBA2) {
-                    const int b = tile / H, bg = b * p.G + (tile - b * H) / hpg;
+                    if (i > 0 && ++hl == hpg) {
+                        hl = 0;
+                        ++bg;
+                    }
                     if (bg != cur_bg) {
                         load_vec_frag<KS>(bh, bl, p.rec + (size_t)bg * gfl, CC, npos, lane);
                         cur_bg = bg;
@@ -349,32 +362,66 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
                 const size_t y_off = (size_t)tile * R;
                 const int g = lane >> 2, t = lane & 3;
                 for (int mb = wt; mb < MB; mb += kTeamWarps) {
-                    float d[4] = {0.f, 0.f, 0.f, 0.f};
                     // ldmatrix rows: lane l addresses row (l & 7) + 8 ((l >> 3) & 1) of the block, chunk l >> 4
                     int lr = mb * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
                     lr = lr < R ? lr : R - 1;   // rows past the tile repeat its last row; their results are dropped
                     const int rr = i * R + lr;
+                    uint32_t a[KS][4];
+#pragma unroll
+                    for (int ks = 0; ks < KS; ++ks) ldmatrix_x4(a[ks], chunk_at(st, rr, ks * 2 + (lane >> 4)));
+                    // four independent accumulation chains: (k-step parity) x (high, low part)
+                    float d[4][4];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+#pragma unroll
+                        for (int f = 0; f < 4; ++f) d[c][f] = 0.f;
 #pragma unroll
                     for (int ks = 0; ks < KS; ++ks) {
-                        uint32_t a[4];
-                        ldmatrix_x4(a, chunk_at(st, rr, ks * 2 + (lane >> 4)));
-                        mma_bf16(d, a, bh[ks][0], bh[ks][1]);
-                        mma_bf16(d, a, bl[ks][0], bl[ks][1]);
+                        mma_bf16(d[(ks & 1) * 2], a[ks], bh[ks][0], bh[ks][1]);
+                        mma_bf16(d[(ks & 1) * 2 + 1], a[ks], bl[ks][0], bl[ks][1]);
                     }
-                    // d[0], d[1]: row g, positions 2t, 2t + 1; d[2], d[3]: row g + 8
+                    // buffer terms of rows g and g + 8, entries split over the lane quad
+                    const int row0 = mb * 16 + g, row1 = row0 + 8;
+                    float zq[2][NP];
+#pragma unroll
+                    for (int hr = 0; hr < 2; ++hr)
+#pragma unroll
+                        for (int j = 0; j < NP; ++j) zq[hr][j] = 0.f;
+                    for (int e = t; e < Lr; e += 4) {
+                        const size_t wrow = (size_t)((hs + e) & p.cap_mask) * R;
+                        const float w0 = row0 < R ? lds_in(wblk, wrow + row0, p.in_dtype) : 0.f;
+                        const float w1 = row1 < R ? lds_in(wblk, wrow + row1, p.in_dtype) : 0.f;
+#pragma unroll
+                        for (int j = 0; j < NP; ++j) {
+                            if (j >= npos) break;
+                            const float c = coef[j * cap + e];
+                            zq[0][j] = fmaf(c, w0, zq[0][j]);
+                            zq[1][j] = fmaf(c, w1, zq[1][j]);
+                        }
+                    }
+#pragma unroll
+                    for (int hr = 0; hr < 2; ++hr)
+#pragma unroll
+                        for (int j = 0; j < NP; ++j) {
+                            zq[hr][j] += __shfl_xor_sync(0xffffffffu, zq[hr][j], 1);
+                            zq[hr][j] += __shfl_xor_sync(0xffffffffu, zq[hr][j], 2);
+                        }
+                    // fragment f = 2 hr + hc: row g + 8 hr, position 2t + hc
 #pragma unroll
                     for (int hr = 0; hr < 2; ++hr) {
-                        const int row = mb * 16 + g + 8 * hr;
+                        const int row = hr ? row1 : row0;
                         if (row >= R) continue;
 #pragma unroll
                         for (int hc = 0; hc < 2; ++hc) {
                             const int j = 2 * t + hc;
                             if (j >= npos) continue;
                             float z = 0.f;
-                            for (int e = 0; e < Lr; ++e)
-                                z = fmaf(coef[j * cap + e],
-                                         lds_in(wblk, (size_t)((hs + e) & p.cap_mask) * R + row, p.in_dtype), z);
-                            st_out(y, y_off + j * y_pos_stride + row, fmaf(mul[j], d[2 * hr + hc], z), p.out_dtype);
+#pragma unroll
+                            for (int jj = 0; jj < NP; ++jj)
+                                if (jj == j) z = zq[hr][jj];
+                            const int f = 2 * hr + hc;
+                            const float dot = (d[0][f] + d[2][f]) + (d[1][f] + d[3][f]);
+                            st_out(y, y_off + j * y_pos_stride + row, fmaf(mul[j], dot, z), p.out_dtype);
                         }
                     }
                 }
@@ -400,11 +447,24 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
         const int niter = (R + GROUPS * RG - 1) / (GROUPS * RG);
         float v[NP][CPT * VEC];
         int cur_bg = -1;   // (sequence, group) whose C vectors v holds (Mamba-2)
+        // With R a multiple of 8 the swizzle of a row depends only on the row
+        // within its tile, so a thread's chunk offsets are the same in every
+        // tile of a single-iteration pass: computed once.
+        const bool fixed_offs = (R & 7) == 0 && niter == 1;
+        uint32_t offs[RG][CPT];
+#pragma unroll
+        for (int r = 0; r < RG; ++r)
+#pragma unroll
+            for (int c = 0; c < CPT; ++c)
+                offs[r][c] = static_cast<uint32_t>(chunk_at(smem, row0 * RG + r, tl + c * TPR) - smem);
         for (int m = 0; m * RL::NT + team < nst; ++m) {
             const int k = m * RL::NT + team, s = team * SPT + m % SPT, u = m / SPT;
             const int first = t0 + k * TT, cnt = nt - k * TT < TT ? nt - k * TT : TT;
+            int bg = 0, hl = 0;   // as in the tensor-core path
             if (KIND == RS_MAMBA2) {   // issued before the wait, so the load overlaps it
-                const int b = first / H, bg = b * p.G + (first - b * H) / hpg;
+                const int b = first / H, h = first - b * H, g = h / hpg;
+                bg = b * p.G + g;
+                hl = h - g * hpg;
                 if (bg != cur_bg) {
                     load_vec<NP, CPT, VEC, TPR>(v, p.rec + (size_t)bg * gfl, CC, npos, tl);
                     cur_bg = bg;
@@ -423,7 +483,10 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
                 const int Lr = min(max(__float_as_int(mul[kRecLen]), 0), cap);
                 const float *coef = mul + kRecHdr;
                 if (KIND == RS_MAMBA2) {
-                    const int b = tile / H, bg = b * p.G + (tile - b * H) / hpg;
+                    if (i > 0 && ++hl == hpg) {
+                        hl = 0;
+                        ++bg;
+                    }
                     if (bg != cur_bg) {
                         load_vec<NP, CPT, VEC, TPR>(v, p.rec + (size_t)bg * gfl, CC, npos, tl);
                         cur_bg = bg;
@@ -444,7 +507,9 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
                         for (int c = 0; c < CPT; ++c) {
                             raw[r][c] = make_uint4(0u, 0u, 0u, 0u);
                             if (rbase + r < R)
-                                raw[r][c] = *reinterpret_cast<const uint4 *>(chunk_at(st, i * R + rbase + r, tl + c * TPR));
+                                raw[r][c] = *reinterpret_cast<const uint4 *>(
+                                    fixed_offs ? st + (size_t)i * R * BOXB + offs[r][c]
+                                               : chunk_at(st, i * R + rbase + r, tl + c * TPR));
                         }
                     // even / odd columns accumulate in the two halves of packed fp32 FMAs
                     float2 acc2[NP][RG];
