@@ -38,7 +38,7 @@ TRAFFIC = None
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2048)
+    ap.add_argument("--steps", type=int, default=4096)
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", default="rs", choices=["rs", "reference"])
     ap.add_argument("--prefill", type=int, default=PREFILL)
@@ -59,56 +59,65 @@ def peaks():
 # ------------------------------------------------------------- clocks ------
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons through NVML while running."""
+    """Samples the SM clock and the clock-event (throttle) reasons while the
+    timed region runs, with `nvidia-smi -lms` in a child process (a Python
+    thread would hardly run while the main thread issues launches).  The
+    first sample is awaited before the region starts."""
 
-    def __init__(self, index=0, period=0.01):
-        self.samples, self.reasons, self.period = [], set(), period
-        self.stop_ev = threading.Event()
-        self.ok = False
-        try:
-            import pynvml
-            pynvml.nvmlInit()
-            self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
-            self.ok = True
-        except Exception:
-            self.max_mhz = None
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def _run(self):
-        nv = self.nv
-        names = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
-                 "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
-        while not self.stop_ev.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
-                get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
-                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
-                r = get(self.h)
-                for n, bit in names.items():
-                    if r & bit:
-                        self.reasons.add(n)
-            except Exception:
-                pass
-            time.sleep(self.period)
+    def __init__(self, index=0, period_ms=20):
+        self.index, self.period_ms = index, period_ms
+        self.rows, self.max_mhz, self.proc = [], None, None
 
     def __enter__(self):
-        if self.ok:
-            self.t = threading.Thread(target=self._run, daemon=True)
-            self.t.start()
+        import shutil
+        import subprocess
+        exe = shutil.which("nvidia-smi")
+        if exe is None:
+            return self
+        self.proc = subprocess.Popen(
+            [exe, f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+             f"-lms={self.period_ms}"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        self._reader = threading.Thread(target=self._read, daemon=True)
+        self._reader.start()
+        t0 = time.time()
+        while not self.rows and time.time() - t0 < 10 and self.proc.poll() is None:
+            time.sleep(0.005)
+        self.rows.clear()   # samples from here on fall in the timed region
         return self
 
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == 9:
+                self.rows.append(parts)
+
     def __exit__(self, *a):
-        if self.ok:
-            self.stop_ev.set()
-            self.t.join()
+        if self.proc is not None:
+            time.sleep(2 * self.period_ms / 1000)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
 
     def summary(self):
-        if not self.ok or not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-                    "samples": len(self.samples)}
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        mhz, reasons = [], set()
+        for r in list(self.rows):
+            try:
+                mhz.append(float(r[1]))
+                self.max_mhz = float(r[2])
+            except ValueError:
+                continue
+            for name, flag in zip(self.NAMES, r[5:9]):
+                if flag.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(mhz)}
 
 
 # ------------------------------------------------------------ CPU oracle ---
@@ -177,6 +186,32 @@ def reference_arm(args, rank):
     print(json.dumps(line), flush=True)
 
 
+# --------------------------------------------------------- rank helpers ----
+# One process per GPU; every rank decodes its own batch of sequences (weak
+# scaling).  The only cross-rank operations are the timing barrier and the
+# maximum of the ranks' device times.
+
+def rank_seed(rank):
+    """Seed of rank `rank`'s synthetic inputs (distinct sequences per rank)."""
+    return 1 + 1000 * rank
+
+
+def max_over_ranks(x, world, device):
+    """Maximum of a per-rank float over all ranks (the job's time)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world, batch_per_rank, steps, ms):
+    """Whole-job throughput: all ranks' tokens over the slowest rank's time."""
+    return world * batch_per_rank * steps / (ms * 1e-3)
+
+
 # ------------------------------------------------------------- GPU arm -----
 
 def gpu_arm(args, rank, world):
@@ -190,7 +225,7 @@ def gpu_arm(args, rank, world):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
-    seed = 1 + 1000 * rank
+    seed = rank_seed(rank)
 
     A, D, dtb = gen.mamba2_params(H, seed, dev)
     src = gen.Mamba2Stream(B, H, P, N, G, torch.bfloat16, dtb, seed + 10_000, dev)
@@ -252,11 +287,8 @@ def gpu_arm(args, rank, world):
         e1.record(stream)
         torch.cuda.synchronize()
     launches = rs.rs_launch_count() - n0
-    ms = e0.elapsed_time(e1)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
 
     # pass 2: per-kernel durations for the roofline (the library's own events
@@ -319,11 +351,7 @@ def gpu_arm(args, rank, world):
         y_host.copy_(y, non_blocking=True)
     b1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = b0.elapsed_time(b1) / ne2e
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(b0.elapsed_time(b1) / ne2e, world, dev)
 
     status, flags = sess.get_error()
     if status != rs.RS_OK:
@@ -338,7 +366,7 @@ def gpu_arm(args, rank, world):
     com_avg = statistics.mean(com_ms) if com_ms else float("nan")
     commit_bytes = B * H * P * N * (4 + 4 + 2)
     step_ms = ms / args.steps
-    value = world * B * args.steps / (ms * 1e-3)
+    value = job_tokens_per_s(world, B, args.steps, ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
@@ -360,7 +388,7 @@ def gpu_arm(args, rank, world):
                     "step_state_bytes_per_token": H * P * N * (2 + 10 / K_COMMIT),
                     "step_achieved_gbs": B * H * P * N * (2 + 10 / K_COMMIT) / (step_ms * 1e-3) / 1e9},
         "eager": eager,
-        "e2e": {"value": world * B / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": job_tokens_per_s(world, B, 1, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches,
         "clocks": clk.summary(),
