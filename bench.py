@@ -31,8 +31,9 @@ METRIC = "SSM-layer decode tokens/s at batch 256; achieved HBM GB/s vs B200 peak
 UNIT = "tokens/s"
 WORKLOAD = "mamba2-decode-b256-h80-p64-n128-bf16copy-K8"
 # DRAM bytes (read + write) of one streaming-kernel launch on this workload,
-# from an ncu capture of the current kernel (None when not yet captured).
-TRAFFIC = None
+# from an ncu capture of the current kernel (None when not yet captured):
+# 359,566,592 read + 4,994,304 written (profiles/stream_outputs_mamba2_*.md).
+TRAFFIC = 364560896
 
 
 def parse():
