@@ -70,13 +70,18 @@ __host__ __device__ constexpr uint32_t swizzle_mask_for(int box_bytes) {
     return box_bytes == 128 ? 7u : box_bytes == 64 ? 3u : box_bytes == 32 ? 1u : 0u;
 }
 
-// Tiles per stage: about kStageTarget bytes, at most kMaxTilesPerStage, and
-// no more rows than one box may have.
-__host__ __device__ inline int stage_tiles(int R, size_t row_bytes) {
-    size_t tt = kStageTarget / ((size_t)R * row_bytes);
-    tt = tt < 1 ? 1 : tt > (size_t)kMaxTilesPerStage ? (size_t)kMaxTilesPerStage : tt;
-    const size_t by_rows = (size_t)kMaxBoxRows / (size_t)R;
-    return (int)(tt < by_rows ? tt : by_rows);
+// Tiles per stage: about kStageTarget bytes of checkpoint, tiles plus ring
+// blocks within kStageCap bytes, at most kMaxTilesPerStage, and no more rows
+// than one box may have.
+constexpr size_t kStageCap = 48 * 1024;
+__host__ __device__ inline int stage_tiles(int R, size_t row_bytes, size_t blk_bytes) {
+    const size_t tile = (size_t)R * row_bytes;
+    size_t tt = kStageTarget / tile;
+    const size_t by_cap = kStageCap / (tile + blk_bytes), by_rows = (size_t)kMaxBoxRows / (size_t)R;
+    tt = tt < by_cap ? tt : by_cap;
+    tt = tt < by_rows ? tt : by_rows;
+    tt = tt > (size_t)kMaxTilesPerStage ? (size_t)kMaxTilesPerStage : tt;
+    return (int)(tt < 1 ? 1 : tt);
 }
 
 struct StreamLayout {
@@ -90,7 +95,7 @@ struct StreamLayout {
 __host__ __device__ inline StreamLayout stream_layout(int R, size_t row_bytes, size_t blk_bytes, size_t rec_bytes,
                                                       int nt) {
     StreamLayout l;
-    l.TT = stage_tiles(R, row_bytes);
+    l.TT = stage_tiles(R, row_bytes, blk_bytes);
     l.box_rows = l.TT * R;
     const size_t boxb = (size_t)box_bytes_for((int)row_bytes), nbox = row_bytes / boxb;
     l.box_region = align_up((size_t)l.box_rows * boxb, 1024);
@@ -663,7 +668,7 @@ cudaError_t make_state_map(const Params &p, void *map_out) {
                                              : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const cuuint64_t dims[2] = {(cuuint64_t)p.CC, (cuuint64_t)p.B * p.H * p.R};
     const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-    const cuuint32_t box[2] = {(cuuint32_t)(boxb / eb), (cuuint32_t)(stage_tiles(p.R, row_bytes) * p.R)};
+    const cuuint32_t box[2] = {(cuuint32_t)(boxb / eb), (cuuint32_t)(stage_tiles(p.R, row_bytes, p.blk_r) * p.R)};
     const cuuint32_t estr[2] = {1, 1};
     const CUtensorMapSwizzle swz = boxb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                    : boxb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
