@@ -248,6 +248,18 @@ uint64_t rs_launch_count(void);           /* kernels launched by this library so
 rs_status rs_profile_start(rs_handle h, int max_calls);
 rs_status rs_profile_stop(rs_handle h, int *calls, float *prep_ms, float *stream_ms);
 
+/* rs_decode_outputs with its replay records kept in a fixed library-owned
+ * device array instead of the workspace's scratch region.  The pages have no
+ * counterpart to this call: it exists for callers that must not size or
+ * provide scratch memory.  The array holds RS_STATIC_SCRATCH_BYTES; a handle
+ * whose records need more (rs_layout.scratch_bytes) gets RS_ERR_CAPACITY and
+ * nothing is launched.  No device memory is allocated or freed.  The array is
+ * shared by every handle of the process on a device, so calls that may overlap
+ * in time (other streams, other host threads) race; calls ordered on one
+ * stream do not.  Results equal rs_decode_outputs bit for bit. */
+#define RS_STATIC_SCRATCH_BYTES (16u << 20)
+rs_status rs_decode_outputs_static_scratch(rs_handle h, void *y, rs_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -84,6 +84,7 @@ def _load():
         "rs_clear_error": [vp, vp],
         "rs_read_ptrs": [vp, vp, vp, vp],
         "rs_profile_start": [vp, i32],
+        "rs_decode_outputs_static_scratch": [vp, vp, vp],
         "rs_profile_stop": [vp, vp, vp, vp],
     }
     for name, args in sigs.items():
@@ -174,6 +175,11 @@ def rs_append(h, inputs, T, stream=None):
 
 def rs_decode_outputs(h, y, stream=None):
     _check(_lib.rs_decode_outputs(h, _ptr(y), _stream(stream)), "rs_decode_outputs")
+
+
+def rs_decode_outputs_static_scratch(h, y, stream=None):
+    _check(_lib.rs_decode_outputs_static_scratch(h, _ptr(y), _stream(stream)),
+           "rs_decode_outputs_static_scratch")
 
 
 def rs_decode_step(h, inputs, T, y, stream=None):

@@ -336,6 +336,38 @@ rs_status rs_decode_step(rs_handle h, const rs_inputs *in, int T, void *y, rs_st
                     "decode_step", 2);
 }
 
+namespace {
+
+// Replay records of rs_decode_outputs_static_scratch: a fixed device array, its
+// address looked up once per device.
+__device__ __align__(256) float g_static_scratch[RS_STATIC_SCRATCH_BYTES / sizeof(float)];
+std::atomic<float *> g_static_scratch_ptr[64];
+
+}  // namespace
+
+rs_status rs_decode_outputs_static_scratch(rs_handle h, void *y, rs_stream stream) {
+    if (!h || !y) return RS_ERR_ARG;
+    if (h->lay.scratch_bytes > RS_STATIC_SCRATCH_BYTES) return RS_ERR_CAPACITY;
+    if (h->device < 0 || h->device >= 64) return RS_ERR_UNSUPPORTED;
+    int cur = -1;
+    const cudaError_t ce = cudaGetDevice(&cur);
+    if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
+    if (cur != h->device) return RS_ERR_ARG;   // the array's address is per device
+    float *rec = g_static_scratch_ptr[h->device].load();
+    if (!rec) {
+        void *addr = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&addr, g_static_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+        rec = static_cast<float *>(addr);
+        g_static_scratch_ptr[h->device].store(rec);
+    }
+    rs::Params p = h->p;   // the handle's parameters with the records moved
+    p.rec = rec;
+    const rs_inputs none{};
+    return launched(rs::launch_outputs(p, h->state_map, 1, 0, none, y, static_cast<cudaStream_t>(stream)),
+                    "outputs_static_scratch", 2);
+}
+
 rs_status rs_verify_outputs(rs_handle h, int npos, void *y, rs_stream stream) {
     if (!h || !y) return RS_ERR_ARG;
     if (npos < 1 || npos > h->cfg.npos_max) return RS_ERR_CAPACITY;
