@@ -189,7 +189,7 @@ struct RowCopy {
 };
 
 template <int CC, int NP>
-__global__ void __launch_bounds__(32 * kPrepWarps)
+__global__ void __launch_bounds__(32 * kPrepWarps, (NP <= 2 ? 3 : 1))
 m2_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
     extern __shared__ __align__(16) float psm[];
     allow_dependent_launch();
@@ -466,6 +466,21 @@ gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
                          : static_cast<const void *>(static_cast<const unsigned char *>(inp) +
                                                      (((size_t)(i - L_old) * Bn + b) * H + h) * row);
     };
+    // A decode step's new q and v rows, read now so that the append below does
+    // not wait for them: 8-byte pieces, up to 4 per lane (rows of <= 1 KB).
+    const bool pre_qv = T == 1 && has_head && rowC % 256 == 0 && rowR % 256 == 0 && rowC <= 1024 &&
+                        rowR <= 1024 && ((reinterpret_cast<uintptr_t>(in.q) | reinterpret_cast<uintptr_t>(in.v)) & 7) == 0;
+    uint2 qv[2][4];
+    if (pre_qv) {
+        const size_t at = (size_t)b * H + h;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (u * 256 < (int)rowC)
+                qv[0][u] = reinterpret_cast<const uint2 *>(static_cast<const unsigned char *>(in.q) + at * rowC)[lane + 32 * u];
+            if (u * 256 < (int)rowR)
+                qv[1][u] = reinterpret_cast<const uint2 *>(static_cast<const unsigned char *>(in.v) + at * rowR)[lane + 32 * u];
+        }
+    }
     if (has_head) {
         // ---- one round of asynchronous copies
         for (int i = 0; i < L; ++i) stage_row(kraw + (size_t)i * rowC, src_row(kblk, in.k, rowC, i), (int)rowC, lane, 32);
@@ -546,16 +561,33 @@ gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
                 const int slot = (tail + t) & p.cap_mask;
                 const size_t at = ((size_t)t * Bn + b) * H + h;
                 copy_row(kblk + (size_t)slot * rowC, kraw + (size_t)(L_old + t) * rowC, (int)rowC, lane, 32);
-                copy_row(qblk + (size_t)slot * rowC, static_cast<const unsigned char *>(in.q) + at * rowC, (int)rowC, lane, 32);
-                copy_row(vblk + (size_t)slot * rowR, static_cast<const unsigned char *>(in.v) + at * rowR, (int)rowR, lane, 32);
+                if (pre_qv) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        if (u * 256 < (int)rowC) reinterpret_cast<uint2 *>(qblk + (size_t)slot * rowC)[lane + 32 * u] = qv[0][u];
+                        if (u * 256 < (int)rowR) reinterpret_cast<uint2 *>(vblk + (size_t)slot * rowR)[lane + 32 * u] = qv[1][u];
+                    }
+                } else {
+                    copy_row(qblk + (size_t)slot * rowC, static_cast<const unsigned char *>(in.q) + at * rowC, (int)rowC, lane, 32);
+                    copy_row(vblk + (size_t)slot * rowR, static_cast<const unsigned char *>(in.v) + at * rowR, (int)rowR, lane, 32);
+                }
             }
             for (int t = lane; t < T; t += 32) {
                 ablk[(tail + t) & p.cap_mask] = alpha[L_old + t];
                 bblk[(tail + t) & p.cap_mask] = beta[L_old + t];
             }
+            // the last of the sequence's H warps to get here advances the tail
+            // (every warp has read the pointers before it arrives)
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence();
+                if (atomicAdd(&p.arrive[b], 1u) == static_cast<unsigned>(H - 1)) {
+                    p.arrive[b] = 0u;
+                    p.tail[b] = tail + T;
+                }
+            }
         }
     }
-    if (T > 0) arrive_and_advance(p, b, tail, T, cps);
     if (!ok && T == 0 && hc == 0 && threadIdx.x == 0) atomicOr(&p.err[b], RS_SEQ_ERR_EMPTY);
 }
 

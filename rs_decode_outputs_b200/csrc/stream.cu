@@ -55,11 +55,15 @@ constexpr size_t kStageTarget = 32 * 1024;      // checkpoint bytes a stage aims
 constexpr int kMaxTilesPerStage = 8;
 constexpr int kMaxBoxRows = 256;                // tensor-map box height limit
 
-template <int NP>
+// Consumer teams: 3, except 2 for the CUDA-core contraction of many positions
+// (its register tile needs more than the 128 registers three teams allow).
+__host__ __device__ constexpr bool use_mma(int state_bytes, int NP) { return state_bytes == 2 && NP >= 2; }
+
+template <int NP, bool MMA>
 struct Roles {
-    static constexpr int NT = NP <= 2 ? 3 : 2;        // consumer teams
-    static constexpr int NCW = NT * kTeamWarps;       // consumer warps
-    static constexpr int THREADS = 32 * (NCW + 1);    // + the producer warp
+    static constexpr int NT = (NP <= 2 || MMA) ? 3 : 2;   // consumer teams
+    static constexpr int NCW = NT * kTeamWarps;          // consumer warps
+    static constexpr int THREADS = 32 * (NCW + 1);       // + the producer warp
 };
 
 // Width of the boxes a checkpoint row is copied in, and the matching swizzle:
@@ -206,12 +210,12 @@ __device__ __forceinline__ void load_vec_frag(uint32_t (&bh)[KS][2], uint32_t (&
 }
 
 template <int KIND, int CC, typename TS, int NP>
-__global__ void __launch_bounds__(Roles<NP>::THREADS, 1)
+__global__ void __launch_bounds__((Roles<NP, use_mma(TS::bytes, NP)>::THREADS), 1)
 stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, int npos, void *y) {
-    using RL = Roles<NP>;
+    using RL = Roles<NP, use_mma(TS::bytes, NP)>;
     constexpr int ROWB = CC * TS::bytes, BOXB = box_bytes_for(ROWB), NBOX = ROWB / BOXB, CPB = BOXB / 16;
     constexpr uint32_t SWM = swizzle_mask_for(BOXB);
-    constexpr bool USE_MMA = TS::bytes == 2 && NP >= 2;   // bf16 copy, several positions: tensor cores
+    constexpr bool USE_MMA = use_mma(TS::bytes, NP);   // bf16 copy, several positions: tensor cores
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int R = p.R, H = p.H, cap = p.cap;
@@ -643,7 +647,8 @@ static int state_bytes(const Params &p) { return p.copy_dtype == RS_BF16 ? 2 : p
 
 static StreamLayout layout_for(const Params &p, int npos) {
     const int NPr = prep_np(npos);
-    const int nt = NPr <= 2 ? Roles<1>::NT : Roles<8>::NT;
+    const bool mma = use_mma(state_bytes(p), NPr);
+    const int nt = NPr <= 2 ? Roles<1, false>::NT : mma ? Roles<8, true>::NT : Roles<8, false>::NT;
     return stream_layout(p.R, (size_t)p.CC * state_bytes(p), p.blk_r, 4 * tile_rec_floats(p.kind, NPr, p.cap, p.CC), nt);
 }
 
@@ -692,7 +697,7 @@ static cudaError_t launch_stream_t(const Params &p, const CUtensorMap &smap, int
     // may start while the prep kernel before it is still running (see grid_dependency_wait)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(Roles<NP>::THREADS);
+    cfg.blockDim = dim3(Roles<NP, use_mma(TS::bytes, NP)>::THREADS);
     cfg.dynamicSmemBytes = lay.total;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
