@@ -157,6 +157,14 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t (&a)[4], const void *smem_r
                  : "r"(smem_u32(smem_row)));
 }
 
+// The same from a k-major store: each lane addresses one 16-byte row of a
+// transposed 8x8 block, and receives the fragment of the transpose.
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&a)[4], const void *smem_row) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+                 : "r"(smem_u32(smem_row)));
+}
+
 // D += A B for one m16n8k16 bf16 tile with fp32 accumulation.
 __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
@@ -328,6 +336,13 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
         const int MB = (R + 15) / 16;       // 16-row blocks of a tile
         uint32_t bh[KS][2], bl[KS][2];
         int cur_bg = -1;
+        // The buffer terms sum_i coef_j[i] w_i[r] are a product too: rows r of
+        // the ring block (k = ring slot) times the coefficients moved to slot
+        // order, in up to two more k-steps with their own accumulators (the
+        // multiplier mul_j scales only the checkpoint part).  bf16 rings of up
+        // to 32 slots with R a multiple of 8; otherwise summed per lane below.
+        const bool zmma = p.in_dtype == RS_BF16 && cap <= 32 && (R & 7) == 0;
+        const int KE = (cap + 15) / 16;
         for (int m = 0; m * RL::NT + team < nst; ++m) {
             const int k = m * RL::NT + team, s = team * SPT + m % SPT, u = m / SPT;
             const int first = t0 + k * TT, cnt = nt - k * TT < TT ? nt - k * TT : TT;
@@ -370,6 +385,24 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
                 }
                 const size_t y_off = (size_t)tile * R;
                 const int g = lane >> 2, t = lane & 3;
+                // B fragments of the buffer terms: coef_n[e(s)] at slots s = 16 kse + 2t + {0, 1} (+ 8),
+                // e(s) = (s - head slot) mod cap, zero where e(s) >= L, s >= cap or n >= npos
+                uint32_t zh[2][2], zl[2][2];
+                if (zmma) {
+#pragma unroll
+                    for (int kse = 0; kse < 2; ++kse)
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            float cv[2];
+#pragma unroll
+                            for (int q = 0; q < 2; ++q) {
+                                const int sl = kse * 16 + 2 * t + 8 * hh + q;
+                                const int e = (sl - hs) & p.cap_mask;
+                                cv[q] = (g < npos && sl < cap && e < Lr) ? coef[g * cap + e] : 0.f;
+                            }
+                            split_bf16x2(cv[0], cv[1], zh[kse][hh], zl[kse][hh]);
+                        }
+                }
                 for (int mb = wt; mb < MB; mb += kTeamWarps) {
                     // ldmatrix rows: lane l addresses row (l & 7) + 8 ((l >> 3) & 1) of the block, chunk l >> 4
                     int lr = mb * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
@@ -389,14 +422,38 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
                         mma_bf16(d[(ks & 1) * 2], a[ks], bh[ks][0], bh[ks][1]);
                         mma_bf16(d[(ks & 1) * 2 + 1], a[ks], bl[ks][0], bl[ks][1]);
                     }
-                    // buffer terms of rows g and g + 8, entries split over the lane quad
                     const int row0 = mb * 16 + g, row1 = row0 + 8;
+                    float dz[4] = {0.f, 0.f, 0.f, 0.f};   // buffer terms, fragment layout (zmma)
+                    if (zmma) {
+                        float d2[2][4];
+#pragma unroll
+                        for (int c = 0; c < 2; ++c)
+#pragma unroll
+                            for (int f = 0; f < 4; ++f) d2[c][f] = 0.f;
+                        // transposed 8x8 blocks of the ring block: lane l reads slot 8 ((l >> 4) & 1) + (l & 7)
+                        // of the k-step, rows r0 .. r0 + 7 with r0 = 16 mb + 8 ((l >> 3) & 1)
+                        int r0 = mb * 16 + ((lane >> 3) & 1) * 8;
+                        r0 = r0 + 8 <= R ? r0 : R - 8;   // stays inside the block; rows >= R are dropped
+#pragma unroll
+                        for (int kse = 0; kse < 2; ++kse) {
+                            if (kse >= KE) break;
+                            int sl = kse * 16 + ((lane >> 4) & 1) * 8 + (lane & 7);
+                            sl = sl < cap ? sl : 0;   // padding slots read row 0; their coefficients are 0
+                            uint32_t a[4];
+                            ldmatrix_x4_trans(a, wblk + ((size_t)sl * R + r0) * 2);
+                            mma_bf16(d2[0], a, zh[kse][0], zh[kse][1]);
+                            mma_bf16(d2[1], a, zl[kse][0], zl[kse][1]);
+                        }
+#pragma unroll
+                        for (int f = 0; f < 4; ++f) dz[f] = d2[0][f] + d2[1][f];
+                    }
+                    // otherwise: buffer terms of rows g and g + 8, entries split over the lane quad
                     float zq[2][NP];
 #pragma unroll
                     for (int hr = 0; hr < 2; ++hr)
 #pragma unroll
                         for (int j = 0; j < NP; ++j) zq[hr][j] = 0.f;
-                    for (int e = t; e < Lr; e += 4) {
+                    for (int e = zmma ? Lr : t; e < Lr; e += 4) {
                         const size_t wrow = (size_t)((hs + e) & p.cap_mask) * R;
                         const float w0 = row0 < R ? lds_in(wblk, wrow + row0, p.in_dtype) : 0.f;
                         const float w1 = row1 < R ? lds_in(wblk, wrow + row1, p.in_dtype) : 0.f;
@@ -424,11 +481,11 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
                         for (int hc = 0; hc < 2; ++hc) {
                             const int j = 2 * t + hc;
                             if (j >= npos) continue;
-                            float z = 0.f;
+                            const int f = 2 * hr + hc;
+                            float z = dz[f];
 #pragma unroll
                             for (int jj = 0; jj < NP; ++jj)
-                                if (jj == j) z = zq[hr][jj];
-                            const int f = 2 * hr + hc;
+                                if (jj == j) z += zq[hr][jj];
                             const float dot = (d[0][f] + d[2][f]) + (d[1][f] + d[3][f]);
                             st_out(y, y_off + j * y_pos_stride + row, fmaf(mul[j], dot, z), p.out_dtype);
                         }
