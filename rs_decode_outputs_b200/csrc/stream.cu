@@ -77,7 +77,7 @@ __host__ __device__ constexpr uint32_t swizzle_mask_for(int box_bytes) {
 // Tiles per stage: about kStageTarget bytes of checkpoint, tiles plus ring
 // blocks within kStageCap bytes, at most kMaxTilesPerStage, and no more rows
 // than one box may have.
-constexpr size_t kStageCap = 48 * 1024;
+constexpr size_t kStageCap = 36 * 1024;
 __host__ __device__ inline int stage_tiles(int R, size_t row_bytes, size_t blk_bytes) {
     const size_t tile = (size_t)R * row_bytes;
     size_t tt = kStageTarget / tile;
