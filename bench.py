@@ -168,8 +168,13 @@ def reference_arm(args, rank):
     if rank != 0:
         return
     cores = os.cpu_count() or 1
-    s = OracleSample(4, 4, 0)
-    s.run(cores)
+    # each step: nseq sequences x all heads x 8 decode steps, nseq sized (<= 32)
+    # so that the whole warm-up + timed run takes about 90 s of wall time
+    probe = OracleSample(32, 8, 0)
+    probe.run(cores)
+    t32 = probe.run(cores)
+    nseq = int(max(1, min(32, 32 * 90.0 / max((args.steps + args.warmup) * t32, 1e-9))))
+    s = OracleSample(nseq, 8, 0)
     for _ in range(args.warmup):
         s.run(cores)
     el = sum(s.run(cores) for _ in range(args.steps))
