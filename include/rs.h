@@ -237,6 +237,14 @@ const char *rs_status_string(int status);
 const char *rs_last_cuda_error(void);     /* text of the last failing CUDA call */
 uint64_t rs_launch_count(void);           /* kernels launched by this library so far */
 
+/* Failure-detection check, no handle needed: one device thread waits, with
+ * the bounded wait every on-device wait of the library uses, on a barrier
+ * phase that nothing completes, gives up after limit_cycles (1 .. the
+ * library's own limit, 2e9 cycles) and writes, into result (device, uint32
+ * [3]): RS_SEQ_ERR_TIMEOUT, then the cycles it waited (low, high words).  The
+ * context stays usable.  RS_ERR_ARG for a NULL result or a limit out of range. */
+rs_status rs_selftest_bounded_wait(uint32_t *result, long long limit_cycles, rs_stream stream);
+
 /* Kernel timing of the output calls (rs_decode_outputs, rs_verify_outputs,
  * rs_decode_step), which each run a small prep kernel and one streaming
  * kernel.  rs_profile_start creates CUDA events for the next `max_calls`

@@ -84,6 +84,7 @@ def _load():
         "rs_clear_error": [vp, vp],
         "rs_read_ptrs": [vp, vp, vp, vp],
         "rs_profile_start": [vp, i32],
+        "rs_selftest_bounded_wait": [vp, ctypes.c_longlong, vp],
         "rs_decode_outputs_static_scratch": [vp, vp, vp],
         "rs_profile_stop": [vp, vp, vp, vp],
     }
@@ -254,3 +255,8 @@ def rs_profile_stop(h):
     _check(_lib.rs_profile_stop(h, ctypes.byref(n), ctypes.byref(tp), ctypes.byref(ts)),
            "rs_profile_stop")
     return n.value, tp.value, ts.value
+
+
+def rs_selftest_bounded_wait(result, limit_cycles, stream=None):
+    _check(_lib.rs_selftest_bounded_wait(_ptr(result), int(limit_cycles), _stream(stream)),
+           "rs_selftest_bounded_wait")

@@ -368,6 +368,12 @@ rs_status rs_decode_outputs_static_scratch(rs_handle h, void *y, rs_stream strea
                     "outputs_static_scratch", 2);
 }
 
+rs_status rs_selftest_bounded_wait(uint32_t *result, long long limit_cycles, rs_stream stream) {
+    if (!result || limit_cycles < 1 || limit_cycles > rs::kWaitLimitCycles) return RS_ERR_ARG;
+    return launched(rs::launch_wait_selftest(result, limit_cycles, static_cast<cudaStream_t>(stream)),
+                    "selftest_bounded_wait");
+}
+
 rs_status rs_verify_outputs(rs_handle h, int npos, void *y, rs_stream stream) {
     if (!h || !y) return RS_ERR_ARG;
     if (npos < 1 || npos > h->cfg.npos_max) return RS_ERR_CAPACITY;

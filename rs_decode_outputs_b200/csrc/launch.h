@@ -71,5 +71,6 @@ cudaError_t launch_load_checkpoint(const Params &p, const float *state, cudaStre
 cudaError_t launch_init(const Params &p, cudaStream_t st);
 cudaError_t launch_eager_accept(const Params &p, int32_t *cur, const int32_t *keep, int nslots,
                                 cudaStream_t st);
+cudaError_t launch_wait_selftest(uint32_t *out, long long limit, cudaStream_t st);
 
 }  // namespace rs

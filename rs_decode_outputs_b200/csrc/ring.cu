@@ -189,4 +189,25 @@ cudaError_t launch_init(const Params &p, cudaStream_t st) {
     return cudaSuccess;
 }
 
+// ------------------------------------------------------ wait self-test ----
+// One thread waits, through the same bounded wait the streaming kernel uses,
+// on a barrier phase that nothing completes; it gives up after `limit` cycles
+// and records RS_SEQ_ERR_TIMEOUT and the cycles it waited.
+__global__ void wait_selftest_kernel(uint32_t *out, long long limit) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    const long long t0 = clock64();
+    const bool done = mbar_wait_bounded(&bar, 0, limit);
+    const long long waited = clock64() - t0;
+    out[0] = done ? 0u : static_cast<uint32_t>(RS_SEQ_ERR_TIMEOUT);
+    out[1] = static_cast<uint32_t>(waited & 0xffffffffLL);
+    out[2] = static_cast<uint32_t>(waited >> 32);
+}
+
+cudaError_t launch_wait_selftest(uint32_t *out, long long limit, cudaStream_t st) {
+    wait_selftest_kernel<<<1, 32, 0, st>>>(out, limit);
+    return cudaGetLastError();
+}
+
 }  // namespace rs
