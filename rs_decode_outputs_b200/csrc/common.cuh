@@ -56,8 +56,6 @@ __device__ __forceinline__ float lds_in(const void *smem_ptr, size_t i, int dtyp
     return static_cast<const float *>(smem_ptr)[i];
 }
 
-__device__ __forceinline__ float lds_f32(const float *smem_ptr, size_t i) { return smem_ptr[i]; }
-
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
@@ -231,34 +229,6 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
     return p;
-}
-
-// Issue the bulk copy of a whole tile in pieces of at most 32 KiB.
-__device__ __forceinline__ void bulk_tile_g2s(void *dst_smem, const void *src, uint32_t bytes,
-                                              uint64_t *bar, uint64_t policy) {
-    mbar_expect_tx(bar, bytes);
-    uint32_t off = 0;
-    while (off < bytes) {
-        uint32_t n = bytes - off < 32768u ? bytes - off : 32768u;
-        bulk_g2s(static_cast<char *>(dst_smem) + off, static_cast<const char *>(src) + off, n, bar,
-                 policy);
-        off += n;
-    }
-}
-
-// 16-byte global load that bypasses L1 and marks the line evict-first in L2.
-__device__ __forceinline__ uint4 ld_stream16(const void *p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.L2::evict_first.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
-__device__ __forceinline__ void st_stream16(void *p, const uint4 &v) {
-    asm volatile("st.global.L1::no_allocate.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x),
-                 "r"(v.y), "r"(v.z), "r"(v.w)
-                 : "memory");
 }
 
 }  // namespace rs

@@ -6,22 +6,6 @@
 
 namespace rs {
 
-// Cooperative copy of nbytes (a multiple of 2) between global buffers, with
-// 16-byte moves when both ends are 16-byte aligned.
-__device__ __forceinline__ void copy_coop(void *dst, const void *src, size_t nbytes) {
-    const uintptr_t a = reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src);
-    if ((a & 15) == 0 && (nbytes & 15) == 0) {
-        for (size_t i = threadIdx.x; i < nbytes / 16; i += blockDim.x)
-            static_cast<uint4 *>(dst)[i] = static_cast<const uint4 *>(src)[i];
-    } else if ((a & 3) == 0 && (nbytes & 3) == 0) {
-        for (size_t i = threadIdx.x; i < nbytes / 4; i += blockDim.x)
-            static_cast<uint32_t *>(dst)[i] = static_cast<const uint32_t *>(src)[i];
-    } else {
-        for (size_t i = threadIdx.x; i < nbytes / 2; i += blockDim.x)
-            static_cast<uint16_t *>(dst)[i] = static_cast<const uint16_t *>(src)[i];
-    }
-}
-
 // Copy one row of nbytes (a multiple of 2) with the 32 lanes of a warp, in the
 // widest pieces both ends allow.
 __device__ __forceinline__ void warp_copy(void *dst, const void *src, size_t nbytes, int lane) {
