@@ -97,8 +97,7 @@ gdn_commit_kernel(const Params p, int min_len, const int32_t *__restrict__ mask)
     if (p.copy_dtype != RS_NONE) store_tile(t, p.copy, tile, p.copy_dtype, p.scale, red);
 
     __syncthreads();
-    if (tid == 0) {
-        __threadfence();
+    if (tid == 0) {   // no fence: nothing in this kernel reads head after the CTAs' reads at entry
         if (atomicAdd(&p.arrive[b], 1u) == static_cast<unsigned>(H - 1)) {
             p.arrive[b] = 0u;
             p.head[b] = head + L;

@@ -68,11 +68,13 @@ __device__ __forceinline__ void copy_row(void *dst, const void *src, int bytes, 
     }
 }
 
-// Last arrival of the `ctas` CTAs of sequence b advances its tail by T.
+// Last arrival of the `ctas` CTAs of sequence b advances its tail by T.  No
+// fence: every CTA has read the pointers before it arrives, nothing in this
+// kernel reads the tail or the ring slots it writes, and the next kernel on
+// the stream sees all of this kernel's writes.
 __device__ __forceinline__ void arrive_and_advance(const Params &p, int b, int tail, int T, int ctas) {
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
         if (atomicAdd(&p.arrive[b], 1u) == static_cast<unsigned>(ctas - 1)) {
             p.arrive[b] = 0u;
             p.tail[b] = tail + T;
@@ -427,7 +429,7 @@ __host__ __device__ inline GdnPrepSmem gdn_prep_smem(int cap, int CC, int NP, in
 }
 
 template <int CC, int NP>
-__global__ void __launch_bounds__(32 * kPrepWarps)
+__global__ void __launch_bounds__(32 * kPrepWarps, (NP <= 2 ? 5 : 1))
 gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
     extern __shared__ __align__(16) unsigned char psm_g[];
     allow_dependent_launch();
@@ -577,10 +579,10 @@ gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
                 bblk[(tail + t) & p.cap_mask] = beta[L_old + t];
             }
             // the last of the sequence's H warps to get here advances the tail
-            // (every warp has read the pointers before it arrives)
+            // (every warp has read the pointers before it arrives; no fence, as
+            // in arrive_and_advance)
             __syncwarp();
             if (lane == 0) {
-                __threadfence();
                 if (atomicAdd(&p.arrive[b], 1u) == static_cast<unsigned>(H - 1)) {
                     p.arrive[b] = 0u;
                     p.tail[b] = tail + T;
