@@ -131,8 +131,9 @@ typedef struct {
     size_t scratch, scratch_bytes; /* fp32 replay records, written and read inside one
                                       output call (NP = npos_max rounded up to 1, 2, 5, 8):
                                       Mamba-2: [B][G][NP Cc] group records, then
-                                      [B][H][16 + NP cap] tile records; GDN: [B][H][16 +
-                                      NP (cap + Cc)]; each record rounded up to 16 bytes  */
+                                      [B][H][16 + NP cs] tile records; GDN: [B][H][16 +
+                                      NP (cs + Cc)], cs = cap rounded up to 4, plus 4;
+                                      each record rounded up to 16 bytes                  */
     size_t total;
 } rs_layout;
 

@@ -8,7 +8,7 @@
 //     y_j[r] = mul_j (S0[r, :] . vec_j) + sum_{i<=e_j} coef_j[i] w_i[r]
 // where w_i is the tile's ring row of entry i (Mamba-2 x_i, GDN v_i).
 //
-// Tile record:   hdr [16] | coef [NP][cap] | vec [NP][CC] (GDN only)
+// Tile record:   hdr [16] | coef [NP][coef_stride(cap)] | vec [NP][CC] (GDN only)
 //                hdr[0..7] = mul_j, hdr[8] = head slot, hdr[9] = L (int bits)
 // Group record:  vec [NP][CC]   (Mamba-2: C_{e_j}, one per (sequence, group))
 // All fp32, each record padded to 16 bytes.  NP is the number of output
@@ -29,9 +29,14 @@ __host__ __device__ inline int prep_np(int npos) {
     return npos <= 1 ? 1 : npos <= 2 ? 2 : npos <= 5 ? 5 : 8;
 }
 
+// Row stride (floats) of coef [NP][.] in a tile record: cap rounded up to 4,
+// plus 4, so that the rows of different positions start in different
+// shared-memory banks (they are read 8 rows at a time by the tensor-core path).
+__host__ __device__ inline int coef_stride(int cap) { return (cap + 3) / 4 * 4 + 4; }
+
 // Floats per tile record for NPr compiled positions.
 __host__ __device__ inline size_t tile_rec_floats(int kind, int NPr, int cap, int CC) {
-    return align_up(kRecHdr + (size_t)NPr * cap + (kind == RS_GDN ? (size_t)NPr * CC : 0), 4);
+    return align_up(kRecHdr + (size_t)NPr * coef_stride(cap) + (kind == RS_GDN ? (size_t)NPr * CC : 0), 4);
 }
 
 // Floats per group record (Mamba-2 only).

@@ -206,6 +206,7 @@ m2_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
     float *sA = sdt + (size_t)HC * cap, *sD = sA + HC, *sS = sD + HC;
     float *cum = sS + HC + (size_t)warp * cap;
     const size_t trf = tile_rec_floats(RS_MAMBA2, NP, cap, CC);
+    const int cstr = coef_stride(cap);
     float *grec = p.rec + ((size_t)b * G + g) * group_rec_floats(NP, CC);
     float *trec0 = p.rec + p.rec_tile_off + ((size_t)b * H + h0) * trf;   // the group's heads
     const size_t rowB = (size_t)CC * ib, rowX = (size_t)R * ib;
@@ -345,7 +346,7 @@ m2_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
                         const float ce = __shfl_sync(0xffffffffu, c, e, SW);
                         if (hv && i == 0) trec[j] = expf(A * ce) * tsc;
                         if (hv && i < L)
-                            trec[kRecHdr + j * cap + i] =
+                            trec[kRecHdr + j * cstr + i] =
                                 i <= e ? fmaf(expf(A * (ce - c)) * dv, bc[j * cap + i], i == e ? Dh : 0.f) : 0.f;
                     }
                     if (hv && i == 0) write_header(trec, head, L, p.cap_mask);
@@ -370,7 +371,7 @@ m2_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
                         const float ce = cum[e];
                         if (lane == 0) trec[j] = expf(A * ce) * tsc;
                         for (int i = lane; i < L; i += 32)
-                            trec[kRecHdr + j * cap + i] =
+                            trec[kRecHdr + j * cstr + i] =
                                 i <= e ? fmaf(expf(A * (ce - cum[i])) * dts[i], bc[j * cap + i], i == e ? Dh : 0.f)
                                        : 0.f;
                     }
@@ -498,7 +499,8 @@ gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
         __syncwarp();
 
         if (ok) {
-            float *coef = trec + kRecHdr, *vec = coef + (size_t)NP * cap;
+            const int cstr = coef_stride(cap);
+            float *coef = trec + kRecHdr, *vec = coef + (size_t)NP * cstr;
             const float sc = p.gdn_scale;
             const float tscale = p.copy_dtype == RS_E4M3 ? p.scale[tile] : 1.f;
             constexpr int UPL = (CC + 31) / 32;
@@ -534,11 +536,11 @@ gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
                     if (j >= npos) continue;
                     if (i <= L - npos + j) {
                         const float f = bt * d[j];
-                        if (lane == 0) coef[j * cap + i] = sc * f;
+                        if (lane == 0) coef[j * cstr + i] = sc * f;
 #pragma unroll
                         for (int m = 0; m < UPL; ++m) u[j][m] = a * fmaf(-f, kr[m], u[j][m]);
                     } else if (lane == 0) {
-                        coef[j * cap + i] = 0.f;
+                        coef[j * cstr + i] = 0.f;
                     }
                 }
             }

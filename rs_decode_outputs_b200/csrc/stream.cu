@@ -226,7 +226,7 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
     constexpr bool USE_MMA = use_mma(TS::bytes, NP);   // bf16 copy, several positions: tensor cores
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const int R = p.R, H = p.H, cap = p.cap;
+    const int R = p.R, H = p.H, cap = p.cap, cstr = coef_stride(cap);
     const size_t rfl = tile_rec_floats(KIND, NP, cap, CC);
     const uint32_t rec_bytes = static_cast<uint32_t>(4 * rfl);
     const uint32_t blk_bytes = static_cast<uint32_t>(p.blk_r);
@@ -381,7 +381,7 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
                         cur_bg = bg;
                     }
                 } else {
-                    load_vec_frag<KS>(bh, bl, coef + (size_t)NP * cap, CC, npos, lane);
+                    load_vec_frag<KS>(bh, bl, coef + (size_t)NP * cstr, CC, npos, lane);
                 }
                 const size_t y_off = (size_t)tile * R;
                 const int g = lane >> 2, t = lane & 3;
@@ -398,7 +398,7 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
                             for (int q = 0; q < 2; ++q) {
                                 const int sl = kse * 16 + 2 * t + 8 * hh + q;
                                 const int e = (sl - hs) & p.cap_mask;
-                                cv[q] = (g < npos && sl < cap && e < Lr) ? coef[g * cap + e] : 0.f;
+                                cv[q] = (g < npos && sl < cap && e < Lr) ? coef[g * cstr + e] : 0.f;
                             }
                             split_bf16x2(cv[0], cv[1], zh[kse][hh], zl[kse][hh]);
                         }
@@ -460,7 +460,7 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
 #pragma unroll
                         for (int j = 0; j < NP; ++j) {
                             if (j >= npos) break;
-                            const float c = coef[j * cap + e];
+                            const float c = coef[j * cstr + e];
                             zq[0][j] = fmaf(c, w0, zq[0][j]);
                             zq[1][j] = fmaf(c, w1, zq[1][j]);
                         }
@@ -558,7 +558,7 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
                         cur_bg = bg;
                     }
                 } else {
-                    load_vec<NP, CPT, VEC, TPR>(v, coef + (size_t)NP * cap, CC, npos, tl);
+                    load_vec<NP, CPT, VEC, TPR>(v, coef + (size_t)NP * cstr, CC, npos, tl);
                 }
                 float mj[NP];
 #pragma unroll
@@ -613,7 +613,7 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
                                 const float w = lds_in(wblk, (size_t)((hs + e) & p.cap_mask) * R + row, p.in_dtype);
 #pragma unroll
                                 for (int j = 0; j < NP; ++j)
-                                    if (j < npos) zr[j] = fmaf(coef[j * cap + e], w, zr[j]);
+                                    if (j < npos) zr[j] = fmaf(coef[j * cstr + e], w, zr[j]);
                             }
 #pragma unroll
                         for (int j = 0; j < NP; ++j) zr[j] += __shfl_xor_sync(0xffffffffu, zr[j], 1);
@@ -642,7 +642,7 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
                                 const float w = rbase + r < R ? lds_in(wblk, wrow + rbase + r, p.in_dtype) : 0.f;
 #pragma unroll
                                 for (int j = 0; j < NP; ++j)
-                                    if (j < npos) zr[r][j] = fmaf(coef[j * cap + e], w, zr[r][j]);
+                                    if (j < npos) zr[r][j] = fmaf(coef[j * cstr + e], w, zr[r][j]);
                             }
                         }
                         const bool hi = tl & 8;
@@ -668,7 +668,7 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
                                 const float w = lds_in(wblk, (size_t)((hs + e) & p.cap_mask) * R + rbase, p.in_dtype);
 #pragma unroll
                                 for (int j = 0; j < NP; ++j)
-                                    if (j < npos) zr[j] = fmaf(coef[j * cap + e], w, zr[j]);
+                                    if (j < npos) zr[j] = fmaf(coef[j * cstr + e], w, zr[j]);
                             }
 #pragma unroll
                         for (int j = 0; j < NP; ++j) {
