@@ -191,7 +191,7 @@ struct RowCopy {
 };
 
 template <int CC, int NP>
-__global__ void __launch_bounds__(32 * kPrepWarps, (NP <= 2 ? 3 : 1))
+__global__ void __launch_bounds__(32 * kPrepWarps, (NP <= 2 ? 3 : 2))
 m2_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
     extern __shared__ __align__(16) float psm[];
     allow_dependent_launch();
