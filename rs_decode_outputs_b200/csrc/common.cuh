@@ -131,6 +131,17 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
     return o;
 }
 
+// Two fp32 products in one packed instruction: a * b elementwise.
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+    unsigned long long x, y, r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(y) : "f"(b.x), "f"(b.y));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(x), "l"(y));
+    float2 o;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(o.x), "=f"(o.y) : "l"(r));
+    return o;
+}
+
 // Sum over the TPR lanes that share a row (TPR a power of two <= 8, aligned).
 template <int TPR>
 __device__ __forceinline__ float row_sum(float v) {

@@ -41,8 +41,8 @@ gdn_commit_kernel(const Params p, int min_len, const int32_t *__restrict__ mask)
     const int in_bytes = p.in_dtype == RS_BF16 ? 2 : 4;
     float *s_alpha = reinterpret_cast<float *>(smem);
     float *s_beta = s_alpha + cap;
-    float *s_v = s_beta + cap;  // [cap][R]
-    unsigned char *s_k = smem + align_up(4 * (2 * (size_t)cap + (size_t)cap * R), 16);  // [cap][CC]
+    float *s_v = s_beta + cap;  // [cap][R] fp32
+    float *s_k = reinterpret_cast<float *>(smem + align_up(4 * (2 * (size_t)cap + (size_t)cap * R), 16));  // [cap][CC] fp32
     const int tid = threadIdx.x;
     // this head's ring blocks
     const size_t bh = (size_t)b * H + h;
@@ -61,11 +61,18 @@ gdn_commit_kernel(const Params p, int min_len, const int32_t *__restrict__ mask)
         s_alpha[i] = ablk[slot];
         s_beta[i] = bblk[slot];
     }
+    // k rows as fp32, 16 input bytes per thread and step
     const int kshift = __ffs(CC * in_bytes / 16) - 1;   // 16-byte pieces per row, log2
     for (int q = tid; q < (L << kshift); q += kTileThreads) {
         const int i = q >> kshift, w = q & ((1 << kshift) - 1);
-        const unsigned char *src = kblk + (size_t)((head + i) & p.cap_mask) * CC * in_bytes;
-        reinterpret_cast<uint4 *>(s_k + (size_t)i * CC * in_bytes)[w] = reinterpret_cast<const uint4 *>(src)[w];
+        const uint4 v = reinterpret_cast<const uint4 *>(kblk + (size_t)((head + i) & p.cap_mask) * CC * in_bytes)[w];
+        float *dst = s_k + (size_t)i * CC + w * (16 / in_bytes);
+        if (in_bytes == 2) {
+            reinterpret_cast<float4 *>(dst)[0] = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
+            reinterpret_cast<float4 *>(dst)[1] = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
+        } else {
+            *reinterpret_cast<uint4 *>(dst) = v;
+        }
     }
     for (int i = tid >> 5; i < L; i += kTileThreads / 32) {
         const unsigned char *row = vblk + (size_t)((head + i) & p.cap_mask) * R * in_bytes;
@@ -76,20 +83,30 @@ gdn_commit_kernel(const Params p, int min_len, const int32_t *__restrict__ mask)
     for (int i = 0; i < L; ++i) {
         float kf[T::NE];
 #pragma unroll
-        for (int c = 0; c < T::CPT; ++c)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) kf[c * 4 + e] = ld_in(s_k, (size_t)i * CC + t.col(c) + e, p.in_dtype);
+        for (int c = 0; c < T::CPT; ++c) {
+            const float4 f = *reinterpret_cast<const float4 *>(s_k + (size_t)i * CC + t.col(c));
+            kf[c * 4] = f.x;
+            kf[c * 4 + 1] = f.y;
+            kf[c * 4 + 2] = f.z;
+            kf[c * 4 + 3] = f.w;
+        }
         const float a = s_alpha[i], bt = s_beta[i];
 #pragma unroll
         for (int k = 0; k < NPASS; ++k) {
-            float d = 0.f;
+            float2 d2 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < T::NE; ++e) d = fmaf(t.s[k][e], kf[e], d);
-            d = row_sum<T::TPR>(d);
+            for (int e = 0; e < T::NE; e += 2)
+                d2 = ffma2(make_float2(t.s[k][e], t.s[k][e + 1]), make_float2(kf[e], kf[e + 1]), d2);
+            const float d = row_sum<T::TPR>(d2.x + d2.y);
             const float vr = t.valid(k) ? s_v[(size_t)i * R + t.row(k)] : 0.f;
             const float m = bt * fmaf(-a, d, vr);   // beta v[r] - alpha beta (s . k)
 #pragma unroll
-            for (int e = 0; e < T::NE; ++e) t.s[k][e] = fmaf(a, t.s[k][e], m * kf[e]);
+            for (int e = 0; e < T::NE; e += 2) {   // s <- alpha s + m k
+                const float2 r = ffma2(make_float2(a, a), make_float2(t.s[k][e], t.s[k][e + 1]),
+                                       fmul2(make_float2(m, m), make_float2(kf[e], kf[e + 1])));
+                t.s[k][e] = r.x;
+                t.s[k][e + 1] = r.y;
+            }
         }
     }
 
@@ -106,9 +123,7 @@ gdn_commit_kernel(const Params p, int min_len, const int32_t *__restrict__ mask)
 }
 
 size_t gdn_commit_smem(const Params &p) {
-    const int in_bytes = p.in_dtype == RS_BF16 ? 2 : 4;
-    return align_up(4 * (2 * (size_t)p.cap + (size_t)p.cap * p.R), 16) +
-           (size_t)in_bytes * p.cap * p.CC;
+    return align_up(4 * (2 * (size_t)p.cap + (size_t)p.cap * p.R), 16) + 4 * (size_t)p.cap * p.CC;
 }
 
 template <int CC, int NPASS>
