@@ -230,6 +230,30 @@ __device__ __forceinline__ void cp_async4(void *smem_dst, const void *gsrc) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
                  : "memory");
 }
+// Four 8x8 b16 matrices from shared memory: lanes 8 q .. 8 q + 7 address the
+// eight 16-byte rows of matrix q; lane l receives row l / 4, elements
+// 2 (l % 4) and 2 (l % 4) + 1 of each (the mma.sync fragment layout).
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&a)[4], const void *smem_row) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+                 : "r"(smem_u32(smem_row)));
+}
+
+// The same for two matrices (lanes 0 .. 15 address them).
+__device__ __forceinline__ void ldmatrix_x2(uint32_t (&a)[2], const void *smem_row) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+                 : "=r"(a[0]), "=r"(a[1])
+                 : "r"(smem_u32(smem_row)));
+}
+
+// D += A B for one m16n8k16 bf16 tile with fp32 accumulation.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                 "{%8, %9}, {%0, %1, %2, %3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }

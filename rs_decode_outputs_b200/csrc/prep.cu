@@ -15,7 +15,8 @@
 // GDN:  vec_j = M_1..M_{e_j} q_{e_j}  (M_i = alpha_i (I - beta_i k_i k_i^T)), by the
 //   backward sweep  u <- q_{e_j};  for i = e_j..1: c_i = beta_i (k_i . u);
 //   u <- alpha_i (u - c_i k_i);  mul_j = scale (x tile scale),
-//   coef_j[i] = scale c_i,  w_i = v_i.
+//   coef_j[i] = scale c_i,  w_i = v_i.  Several positions over bf16 inputs take
+//   an equivalent Gram form of the sweep (gdn_gram_records).
 //
 // With T > 0 the kernel also appends the T step inputs (step 2: append the new
 // SSM input to the buffer): the new entries are read straight from the inputs
@@ -414,9 +415,16 @@ m2_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
 // One warp per (sequence, head); a CTA holds kPrepWarps heads of one sequence.
 // Per-warp shared memory (entries compact, buffer index i at row i):
 //   kraw [cap][CC] | qraw [NP][CC] | alpha [cap] | beta [cap]
+//   (Gram form only:) G, upper triangle by columns [cap (cap - 1) / 2] | P [NP][32]
 struct GdnPrepSmem {
-    size_t k, q, alpha, beta, per_warp;
+    size_t k, q, alpha, beta, g, pc, per_warp;
 };
+
+// Several positions over bf16 inputs with at most 32 buffered entries take
+// the Gram form of the backward sweep (gdn_gram_records).
+__host__ __device__ inline bool gdn_gram(int cap, int CC, int NP, int ib) {
+    return NP >= 2 && ib == 2 && cap <= 32 && CC % 16 == 0;
+}
 
 __host__ __device__ inline GdnPrepSmem gdn_prep_smem(int cap, int CC, int NP, int ib) {
     GdnPrepSmem s;
@@ -425,12 +433,182 @@ __host__ __device__ inline GdnPrepSmem gdn_prep_smem(int cap, int CC, int NP, in
     s.q = w;     w = align_up(w + (size_t)NP * CC * ib, 16);
     s.alpha = w; w = align_up(w + 4 * (size_t)cap, 16);
     s.beta = w;  w = align_up(w + 4 * (size_t)cap, 16);
+    s.g = s.pc = w;
+    if (gdn_gram(cap, CC, NP, ib)) {
+        w = align_up(w + 4 * (size_t)(cap * (cap - 1) / 2), 16);
+        s.pc = w;
+        w = align_up(w + 4 * (size_t)NP * 32, 16);
+    }
     s.per_warp = w;
     return s;
 }
 
+// The backward sweep of one head in Gram form.  Write E_j(l) for the product
+// alpha_l ... alpha_{e_j} (1 for l > e_j).  By induction down from u = q_j, the
+// sweep's vector before step i is
+//     u = E_j(i + 1) (q_j - sum_{i<m<=e_j} h_m k_m),   h_m = c_m / E_j(m + 1),
+// so c_i = beta_i (k_i . u) gives
+//     h_i = beta_i (k_i . q_j - sum_{i<m<=e_j} h_m (k_i . k_m)):
+// the decay factors out of the recurrence.  Hence:
+//   1. the dot products first, as two small products on the tensor cores,
+//      G = K K^T (strict upper triangle) and P = K Q^T (bf16 operands staged
+//      in shared memory, fp32 accumulation);
+//   2. the triangular recurrence for h with one lane per entry, all positions
+//      in lockstep (one broadcast per position and step);
+//   3. E_j(l) by a suffix-product scan over the lanes, then
+//      coef_j[i] = scale h_i E_j(i + 1)  and  vec_j = E_j(0) (q_j - sum_m h_m k_m).
+// Requires L <= 32, CC a multiple of 16, 1 <= npos <= NP <= 8, npos <= L.
 template <int CC, int NP>
-__global__ void __launch_bounds__(32 * kPrepWarps, (NP <= 2 ? 5 : 1))
+__device__ __forceinline__ void gdn_gram_records(const unsigned char *kraw, const unsigned char *qraw,
+                                                 const float *alpha, const float *beta, float *gs, float *ps,
+                                                 int L, int npos, int lane, float sc, float *coef, int cstr,
+                                                 float *vec) {
+    constexpr int KS = CC / 16;
+    constexpr unsigned FULL = 0xffffffffu;
+    const int MT = (L + 15) >> 4, NTL = (L + 7) >> 3;   // 16-row and 8-column blocks of G
+    // ---- 1. G and P.  Rows past L repeat row L - 1 (and positions past npos
+    // repeat npos - 1); their results are not stored.
+    float gacc[2][4][4], pacc[2][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+        for (int f = 0; f < 4; ++f) {
+            pacc[mt][f] = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) gacc[mt][nt][f] = 0.f;
+        }
+    }
+    const unsigned char *arow[2] = {kraw + (size_t)min(lane & 15, L - 1) * CC * 2,
+                                    kraw + (size_t)min(16 + (lane & 15), L - 1) * CC * 2};
+    const unsigned char *qrow = qraw + (size_t)min(lane & 7, npos - 1) * CC * 2;
+    const int acol = (lane >> 4) * 16, qcol = ((lane >> 3) & 1) * 16;   // bytes
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+        uint32_t a[2][4];
+        ldmatrix_x4(a[0], arow[0] + ks * 32 + acol);
+        if (MT > 1) {
+            ldmatrix_x4(a[1], arow[1] + ks * 32 + acol);
+        } else {
+#pragma unroll
+            for (int f = 0; f < 4; ++f) a[1][f] = a[0][f];
+        }
+        uint32_t bq[2];
+        ldmatrix_x2(bq, qrow + ks * 32 + qcol);
+        // B of G's column block nt = rows 8 nt .. 8 nt + 7 of K: fragments 0 and 2
+        // (nt even) or 1 and 3 (nt odd) of the A operand of row block nt / 2
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 2 * mt; nt < 4; ++nt)
+                if (mt < MT && nt < NTL)
+                    mma_bf16(gacc[mt][nt], a[mt], a[nt >> 1][nt & 1], a[nt >> 1][2 + (nt & 1)]);
+        mma_bf16(pacc[0], a[0], bq[0], bq[1]);
+        if (MT > 1) mma_bf16(pacc[1], a[1], bq[0], bq[1]);
+    }
+    // accumulator f of lane (g, t): row g + 8 (f / 2), column 2 t + f % 2 of the block
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+        if (mt >= MT) break;
+#pragma unroll
+        for (int f = 0; f < 4; ++f) {
+            const int i = 16 * mt + g + 8 * (f >> 1), j = 2 * t + (f & 1);
+            if (i < L && j < npos) ps[j * 32 + i] = pacc[mt][f];
+        }
+#pragma unroll
+        for (int nt = 2 * mt; nt < 4; ++nt) {
+            if (nt >= NTL) break;
+#pragma unroll
+            for (int f = 0; f < 4; ++f) {
+                const int i = 16 * mt + g + 8 * (f >> 1), m = 8 * nt + 2 * t + (f & 1);
+                if (i < m && m < L) gs[m * (m - 1) / 2 + i] = gacc[mt][nt][f];
+            }
+        }
+    }
+    __syncwarp();
+    // ---- 2. h_i = beta_i (P[j][i] - acc_i), acc_i = sum of h_m G[i][m] over the
+    // entries m > i done so far; lane i owns entry i
+    const float bl = lane < L ? beta[lane] : 0.f;
+    float pj[NP], acc[NP], hv[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+        pj[j] = (j < npos && lane < L) ? ps[j * 32 + lane] : 0.f;
+        acc[j] = 0.f;
+        hv[j] = 0.f;
+    }
+    for (int i = L - 1; i >= 0; --i) {
+        const float gi = lane < i ? gs[i * (i - 1) / 2 + lane] : 0.f;
+#pragma unroll
+        for (int j = 0; j < NP; ++j) {
+            if (j < npos && i <= L - npos + j) {
+                const float hi = __shfl_sync(FULL, bl * (pj[j] - acc[j]), i);
+                acc[j] = fmaf(hi, gi, acc[j]);
+                if (lane == i) hv[j] = hi;
+            }
+        }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < NP; ++j)
+        if (j < npos) ps[j * 32 + lane] = hv[j];   // h of position j, 0 past e_j
+    // ---- 3. decay products and coefficients
+    float e0[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+        e0[j] = 0.f;
+        if (j >= npos) continue;
+        const int e = L - npos + j;
+        float v = 1.f;
+        if (lane <= e) v = alpha[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {   // inclusive suffix product: E_j(lane)
+            const float w = __shfl_down_sync(FULL, v, o);
+            if (lane + o < 32) v *= w;
+        }
+        float nxt = __shfl_down_sync(FULL, v, 1);   // E_j(lane + 1)
+        if (lane == 31) nxt = 1.f;
+        e0[j] = __shfl_sync(FULL, v, 0);
+        if (lane < L) coef[j * cstr + lane] = lane <= e ? sc * hv[j] * nxt : 0.f;
+    }
+    __syncwarp();
+    // vec_j = E_j(0) (q_j - sum_m h_m k_m), lanes over columns
+    constexpr int UPL = (CC + 31) / 32;
+    float va[NP][UPL];
+#pragma unroll
+    for (int j = 0; j < NP; ++j)
+#pragma unroll
+        for (int u = 0; u < UPL; ++u) {
+            const int c = lane + 32 * u;
+            va[j][u] = (j < npos && c < CC) ? lds_in(qraw, (size_t)j * CC + c, RS_BF16) : 0.f;
+        }
+    for (int m = 0; m < L; ++m) {
+        float kr[UPL];
+#pragma unroll
+        for (int u = 0; u < UPL; ++u) {
+            const int c = lane + 32 * u;
+            kr[u] = c < CC ? lds_in(kraw, (size_t)m * CC + c, RS_BF16) : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < NP; ++j) {
+            if (j >= npos) continue;
+            const float hm = ps[j * 32 + m];
+#pragma unroll
+            for (int u = 0; u < UPL; ++u) va[j][u] = fmaf(-hm, kr[u], va[j][u]);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+        if (j >= npos) continue;
+#pragma unroll
+        for (int u = 0; u < UPL; ++u) {
+            const int c = lane + 32 * u;
+            if (c < CC) vec[j * CC + c] = e0[j] * va[j][u];
+        }
+    }
+}
+
+template <int CC, int NP>
+__global__ void __launch_bounds__(32 * kPrepWarps, (NP == 1 ? 5 : NP == 2 ? 3 : 2))
 gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
     extern __shared__ __align__(16) unsigned char psm_g[];
     allow_dependent_launch();
@@ -473,6 +651,18 @@ gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
     // not wait for them: 8-byte pieces, up to 4 per lane (rows of <= 1 KB).
     const bool pre_qv = T == 1 && has_head && rowC % 256 == 0 && rowR % 256 == 0 && rowC <= 1024 &&
                         rowR <= 1024 && ((reinterpret_cast<uintptr_t>(in.q) | reinterpret_cast<uintptr_t>(in.v)) & 7) == 0;
+    // The v rows of the T <= NP new entries of a verification step, read now
+    // too: rows of <= 256 bytes, one 8-byte piece per lane and row.
+    const bool pre_v = NP >= 2 && !pre_qv && T > 1 && T <= NP && has_head && rowR <= 256 && rowR % 8 == 0 &&
+                       (reinterpret_cast<uintptr_t>(in.v) & 7) == 0;
+    uint2 vpre[NP];
+    if (pre_v) {
+#pragma unroll
+        for (int t = 0; t < NP; ++t)
+            if (t < T && lane * 8 < (int)rowR)
+                vpre[t] = reinterpret_cast<const uint2 *>(static_cast<const unsigned char *>(in.v) +
+                                                          (((size_t)t * Bn + b) * H + h) * rowR)[lane];
+    }
     uint2 qv[2][4];
     if (pre_qv) {
         const size_t at = (size_t)b * H + h;
@@ -498,7 +688,18 @@ gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
         cp_async_wait_all();
         __syncwarp();
 
-        if (ok) {
+        if (ok && gdn_gram(cap, CC, NP, ib)) {
+            const int cstr = coef_stride(cap);
+            float *coef = trec + kRecHdr;
+            const float sc = p.gdn_scale;
+            const float tscale = p.copy_dtype == RS_E4M3 ? p.scale[tile] : 1.f;
+            if constexpr (NP >= 2 && CC % 16 == 0)
+                gdn_gram_records<CC, NP>(kraw, qraw, alpha, beta, reinterpret_cast<float *>(wsm + S.g),
+                                         reinterpret_cast<float *>(wsm + S.pc), L, npos, lane, sc, coef, cstr,
+                                         coef + (size_t)NP * cstr);
+            if (lane < npos) trec[lane] = sc * tscale;
+            if (lane == 0) write_header(trec, head, L, p.cap_mask);
+        } else if (ok) {
             const int cstr = coef_stride(cap);
             float *coef = trec + kRecHdr, *vec = coef + (size_t)NP * cstr;
             const float sc = p.gdn_scale;
@@ -572,9 +773,20 @@ gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
                         if (u * 256 < (int)rowR) reinterpret_cast<uint2 *>(vblk + (size_t)slot * rowR)[lane + 32 * u] = qv[1][u];
                     }
                 } else {
-                    copy_row(qblk + (size_t)slot * rowC, static_cast<const unsigned char *>(in.q) + at * rowC, (int)rowC, lane, 32);
-                    copy_row(vblk + (size_t)slot * rowR, static_cast<const unsigned char *>(in.v) + at * rowR, (int)rowR, lane, 32);
+                    // q: the staged row when the outputs covered this entry (T <= npos)
+                    const unsigned char *qsrc = ok && T <= npos
+                                                    ? qraw + (size_t)(npos - T + t) * rowC
+                                                    : static_cast<const unsigned char *>(in.q) + at * rowC;
+                    copy_row(qblk + (size_t)slot * rowC, qsrc, (int)rowC, lane, 32);
+                    if (!pre_v)
+                        copy_row(vblk + (size_t)slot * rowR, static_cast<const unsigned char *>(in.v) + at * rowR, (int)rowR, lane, 32);
                 }
+            }
+            if (pre_v) {
+#pragma unroll
+                for (int t = 0; t < NP; ++t)
+                    if (t < T && lane * 8 < (int)rowR)
+                        reinterpret_cast<uint2 *>(vblk + (size_t)((tail + t) & p.cap_mask) * rowR)[lane] = vpre[t];
             }
             for (int t = lane; t < T; t += 32) {
                 ablk[(tail + t) & p.cap_mask] = alpha[L_old + t];

@@ -151,26 +151,12 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
     return p;
 }
 
-__device__ __forceinline__ void ldmatrix_x4(uint32_t (&a)[4], const void *smem_row) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
-                 : "r"(smem_u32(smem_row)));
-}
-
 // The same from a k-major store: each lane addresses one 16-byte row of a
 // transposed 8x8 block, and receives the fragment of the transpose.
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&a)[4], const void *smem_row) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                  : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
                  : "r"(smem_u32(smem_row)));
-}
-
-// D += A B for one m16n8k16 bf16 tile with fp32 accumulation.
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-                 "{%8, %9}, {%0, %1, %2, %3};"
-                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 // bf16 pair (first value in the low half) rounded to nearest even, and the
