@@ -6,14 +6,16 @@ elements, rings of 2 to 32 slots, rows that are a multiple of 8 but not of
 16 elements, and a row width that takes the per-lane sum.  Each round
 appends npos entries, verifies all npos outputs against the fp64 oracle,
 rolls back a Bernoulli suffix and commits the long sequences, so the ring
-wraps many times."""
+wraps many times.  The GDN prep takes its Gram form for bf16 inputs and rings
+of up to 32 slots and the sequential sweep otherwise (a 64-slot ring, fp32
+inputs): both are covered, the fp32 ones at the fp32 tolerance."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import rs_decode_outputs_b200 as rs
-from tests.harness import TOL_BF16, GdnCase, Mamba2Case, f64, make_session, rel_err
+from tests.harness import TOL_BF16, TOL_F32, GdnCase, Mamba2Case, f64, make_session, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -31,16 +33,21 @@ SHAPES = [
     ("gdn", 128, 64, 1, 32, 5),  # 32 slots
     ("gdn", 32, 128, 1, 4, 3),   # 4 slots
     ("gdn", 24, 64, 1, 16, 5),
+    ("gdn", 64, 64, 1, 64, 5),   # 64 slots: sequential sweep in the prep
 ]
+# fp32 inputs, fp32 checkpoint without a copy (CUDA-core contraction, sequential sweep)
+SHAPES_F32 = [("m2", 32, 64, 2, 8, 5), ("gdn", 32, 64, 1, 8, 5), ("gdn", 48, 32, 1, 16, 8)]
 
 
-def setup(kind, R, CC, G, cap, npos, dev, seed):
+def setup(kind, R, CC, G, cap, npos, dev, seed, in_dtype=rs.RS_BF16, copy=rs.RS_BF16, scale=1.0):
     if kind == "m2":
-        case = Mamba2Case(B, H, R, CC, G, rs.RS_BF16, seed, dev)
-        sess = make_session(rs.RS_MAMBA2, B, H, R, CC, G, cap=cap, npos_max=npos, A=case.A, D=case.D)
+        case = Mamba2Case(B, H, R, CC, G, in_dtype, seed, dev)
+        sess = make_session(rs.RS_MAMBA2, B, H, R, CC, G, cap=cap, npos_max=npos, in_dtype=in_dtype, copy_dtype=copy,
+                            A=case.A, D=case.D)
     else:
-        case = GdnCase(B, H, CC, R, rs.RS_BF16, seed, dev)
-        sess = make_session(rs.RS_GDN, B, H, R, CC, cap=cap, npos_max=npos)
+        case = GdnCase(B, H, CC, R, in_dtype, seed, dev, scale=scale)
+        sess = make_session(rs.RS_GDN, B, H, R, CC, cap=cap, npos_max=npos, in_dtype=in_dtype, copy_dtype=copy,
+                            gdn_scale=scale)
     g = torch.Generator(device=dev).manual_seed(seed)
     state = 0.2 * torch.randn(B, H, R, CC, device=dev, generator=g)
     sess.load_checkpoint(state)
@@ -68,7 +75,20 @@ def advance(case, kind, s, keep):
 @pytest.mark.parametrize("kind,R,CC,G,cap,npos", SHAPES,
                          ids=[f"{k}-R{r}-C{c}-cap{cp}-n{n}" for k, r, c, _, cp, n in SHAPES])
 def test_verify_rounds_across_ring_widths(cuda_device, kind, R, CC, G, cap, npos):
-    case, sess = setup(kind, R, CC, G, cap, npos, cuda_device, seed=700 + R + cap)
+    # GDN with an output scale other than 1, so that coef and mul carry it
+    case, sess = setup(kind, R, CC, G, cap, npos, cuda_device, seed=700 + R + cap, scale=0.75)
+    verify_rounds(case, sess, kind, cap, npos, R, cuda_device, TOL_BF16)
+
+
+@pytest.mark.parametrize("kind,R,CC,G,cap,npos", SHAPES_F32,
+                         ids=[f"{k}-R{r}-C{c}-cap{cp}-n{n}" for k, r, c, _, cp, n in SHAPES_F32])
+def test_verify_rounds_fp32(cuda_device, kind, R, CC, G, cap, npos):
+    case, sess = setup(kind, R, CC, G, cap, npos, cuda_device, seed=900 + R + cap, in_dtype=rs.RS_F32,
+                       copy=rs.RS_NONE)
+    verify_rounds(case, sess, kind, cap, npos, R, cuda_device, TOL_F32)
+
+
+def verify_rounds(case, sess, kind, cap, npos, R, cuda_device, tol):
     rounds = 10
     acc = rs.inputs.acceptance(rounds, B, npos - 1, 0.6, seed=R + cap)
     min_len = cap - npos + 1   # after a commit every length is below this, so npos more entries fit
@@ -87,6 +107,6 @@ def test_verify_rounds_across_ring_widths(cuda_device, kind, R, CC, G, cap, npos
         length[length >= min_len] = 0
         head, tail = sess.read_ptrs()
         assert np.array_equal(tail - head, length), r
-    assert worst <= TOL_BF16, worst
+    assert worst <= tol, worst
     status, flags = sess.get_error()
     assert status == rs.RS_OK and not flags.any()
