@@ -55,13 +55,20 @@ constexpr size_t kStageTarget = 32 * 1024;      // checkpoint bytes a stage aims
 constexpr int kMaxTilesPerStage = 8;
 constexpr int kMaxBoxRows = 256;                // tensor-map box height limit
 
-// Consumer teams: 3, except 2 for the CUDA-core contraction of many positions
-// (its register tile needs more than the 128 registers three teams allow).
+// Consumer teams: 3; 2 for the CUDA-core contraction of many positions (its
+// register tile needs more than the 128 registers three teams allow); 4 for
+// the tensor-core path up to 5 positions and rows of up to 128 columns, whose
+// warps wait mostly on instruction latency (a fourth team measured 5 to 8 %
+// faster than three at 5 positions, with the 96 registers 17 warps allow; 8
+// positions or 256 columns keep three teams and 128 registers).
 __host__ __device__ constexpr bool use_mma(int state_bytes, int NP) { return state_bytes == 2 && NP >= 2; }
+__host__ __device__ constexpr int consumer_teams(int NP, bool mma, int CC) {
+    return (mma && NP <= 5 && CC <= 128) ? 4 : (NP <= 2 || mma) ? 3 : 2;
+}
 
-template <int NP, bool MMA>
+template <int NP, bool MMA, int CC>
 struct Roles {
-    static constexpr int NT = (NP <= 2 || MMA) ? 3 : 2;   // consumer teams
+    static constexpr int NT = consumer_teams(NP, MMA, CC);   // consumer teams
     static constexpr int NCW = NT * kTeamWarps;          // consumer warps
     static constexpr int THREADS = 32 * (NCW + 1);       // + the producer warp
 };
@@ -93,6 +100,7 @@ struct StreamLayout {
     int TT;         // tiles per stage
     int box_rows;   // rows of every box copy (TT R)
     int S, SPT;     // stages in all, stages per team
+    int NT;         // consumer teams in use
 };
 
 // Stage (1024-byte aligned): nbox boxes of TT R rows | TT ring blocks | TT records.
@@ -106,9 +114,12 @@ __host__ __device__ inline StreamLayout stream_layout(int R, size_t row_bytes, s
     l.blk_off = nbox * l.box_region;
     l.rec_off = align_up(l.blk_off + (size_t)l.TT * blk_bytes, 16);
     l.stage_bytes = align_up(l.rec_off + (size_t)l.TT * rec_bytes, 1024);
-    size_t spt = (kStreamSmemMax - kStreamSmemReserve) / l.stage_bytes / nt;
+    const size_t fit = (kStreamSmemMax - kStreamSmemReserve) / l.stage_bytes;   // stages that fit
+    // four teams (the tensor-core path) only where each gets a stage; else three
+    l.NT = (nt == 4 && fit < 4) ? 3 : nt;
+    size_t spt = fit / l.NT;
     spt = spt < 1 ? 1 : spt > 8 ? 8 : spt;
-    l.S = (int)(spt * nt);
+    l.S = (int)(spt * l.NT);
     l.SPT = (int)spt;
     l.bars = (size_t)l.S * l.stage_bytes;
     l.total = l.bars + align_up(16 * (size_t)l.S, 128) + 1024;   // + slack to align the base to 1024
@@ -204,9 +215,9 @@ __device__ __forceinline__ void load_vec_frag(uint32_t (&bh)[KS][2], uint32_t (&
 }
 
 template <int KIND, int CC, typename TS, int NP>
-__global__ void __launch_bounds__((Roles<NP, use_mma(TS::bytes, NP)>::THREADS), 1)
+__global__ void __launch_bounds__((Roles<NP, use_mma(TS::bytes, NP), CC>::THREADS), 1)
 stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, int npos, void *y) {
-    using RL = Roles<NP, use_mma(TS::bytes, NP)>;
+    using RL = Roles<NP, use_mma(TS::bytes, NP), CC>;
     constexpr int ROWB = CC * TS::bytes, BOXB = box_bytes_for(ROWB), NBOX = ROWB / BOXB, CPB = BOXB / 16;
     constexpr uint32_t SWM = swizzle_mask_for(BOXB);
     constexpr bool USE_MMA = use_mma(TS::bytes, NP);   // bf16 copy, several positions: tensor cores
@@ -220,7 +231,7 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
     // ring rows the outputs sum over: Mamba-2 x, GDN v ([B][H][cap][R] blocks)
     const unsigned char *wring = static_cast<const unsigned char *>(KIND == RS_MAMBA2 ? p.ra : p.rc);
     const StreamLayout lay = stream_layout(R, ROWB, blk_bytes, rec_bytes, RL::NT);
-    const int S = lay.S, SPT = lay.SPT, TT = lay.TT;
+    const int S = lay.S, SPT = lay.SPT, TT = lay.TT, NTU = lay.NT;   // NTU <= RL::NT teams in use
     const uint32_t stage_tx_tiles = static_cast<uint32_t>(NBOX * lay.box_rows * BOXB);
     // stage k of this CTA -> team k % NT, the team's m-th stage (m = k / NT),
     // ring slot (k % NT) * SPT + m % SPT, use m / SPT of that slot
@@ -266,14 +277,14 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
             // grid has finished and its writes are visible).
             const int pre = nst < S ? nst : S;
             for (int k = 0; k < pre; ++k) {   // stage k < S: slot k % NT * SPT + k / NT, first use
-                const int s = (k % RL::NT) * SPT + k / RL::NT;
+                const int s = (k % NTU) * SPT + k / NTU;
                 const int first = t0 + k * TT, cnt = nt - k * TT < TT ? nt - k * TT : TT;
                 mbar_expect_tx(full + s, stage_tx_tiles + cnt * (blk_bytes + rec_bytes));
                 copy_tiles(stage(s), first, full + s);
             }
             grid_dependency_wait();
             for (int k = 0; k < pre; ++k) {
-                const int s = (k % RL::NT) * SPT + k / RL::NT;
+                const int s = (k % NTU) * SPT + k / NTU;
                 const int first = t0 + k * TT, cnt = nt - k * TT < TT ? nt - k * TT : TT;
                 copy_side(stage(s), first, cnt, full + s);
             }
@@ -289,7 +300,7 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
                 mbar_expect_tx(full + s, stage_tx_tiles + cnt * (blk_bytes + rec_bytes));
                 copy_side(st, first, cnt, full + s);
                 copy_tiles(st, first, full + s);
-                if (++team == RL::NT) {
+                if (++team == NTU) {
                     team = 0;
                     if (++ms == SPT) {
                         ms = 0;
@@ -304,6 +315,7 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
     // -------------------------------------------------------------- consumers
     // Team `team` (four warps) contracts stages team, team + NT, ...
     const int team = warp / kTeamWarps;
+    if (team >= NTU) return;   // a team the layout has no stages for (see stream_layout)
     const size_t y_pos_stride = (size_t)p.B * H * R;
     const int hpg = p.heads_per_group;
     const size_t gfl = group_rec_floats(NP, CC);
@@ -329,8 +341,8 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
         // to 32 slots with R a multiple of 8; otherwise summed per lane below.
         const bool zmma = p.in_dtype == RS_BF16 && cap <= 32 && (R & 7) == 0;
         const int KE = (cap + 15) / 16;
-        for (int m = 0; m * RL::NT + team < nst; ++m) {
-            const int k = m * RL::NT + team, s = team * SPT + m % SPT, u = m / SPT;
+        for (int m = 0; m * NTU + team < nst; ++m) {
+            const int k = m * NTU + team, s = team * SPT + m % SPT, u = m / SPT;
             const int first = t0 + k * TT, cnt = nt - k * TT < TT ? nt - k * TT : TT;
             // (sequence, group) of the stage's first tile and its head within the
             // group; consecutive tiles advance the head, and the group index
@@ -451,13 +463,15 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
                             zq[1][j] = fmaf(c, w1, zq[1][j]);
                         }
                     }
+                    if (!zmma) {   // (with zmma the sums above are empty)
 #pragma unroll
-                    for (int hr = 0; hr < 2; ++hr)
+                        for (int hr = 0; hr < 2; ++hr)
 #pragma unroll
-                        for (int j = 0; j < NP; ++j) {
-                            zq[hr][j] += __shfl_xor_sync(0xffffffffu, zq[hr][j], 1);
-                            zq[hr][j] += __shfl_xor_sync(0xffffffffu, zq[hr][j], 2);
-                        }
+                            for (int j = 0; j < NP; ++j) {
+                                zq[hr][j] += __shfl_xor_sync(0xffffffffu, zq[hr][j], 1);
+                                zq[hr][j] += __shfl_xor_sync(0xffffffffu, zq[hr][j], 2);
+                            }
+                    }
                     // fragment f = 2 hr + hc: row g + 8 hr, position 2t + hc
 #pragma unroll
                     for (int hr = 0; hr < 2; ++hr) {
@@ -509,8 +523,8 @@ stream_outputs_kernel(const Params p, const __grid_constant__ CUtensorMap smap, 
 #pragma unroll
             for (int c = 0; c < CPT; ++c)
                 offs[r][c] = static_cast<uint32_t>(chunk_at(smem, row0 * RG + r, tl + c * TPR) - smem);
-        for (int m = 0; m * RL::NT + team < nst; ++m) {
-            const int k = m * RL::NT + team, s = team * SPT + m % SPT, u = m / SPT;
+        for (int m = 0; m * NTU + team < nst; ++m) {
+            const int k = m * NTU + team, s = team * SPT + m % SPT, u = m / SPT;
             const int first = t0 + k * TT, cnt = nt - k * TT < TT ? nt - k * TT : TT;
             int bg = 0, hl = 0;   // as in the tensor-core path
             if (KIND == RS_MAMBA2) {   // issued before the wait, so the load overlaps it
@@ -691,7 +705,7 @@ static int state_bytes(const Params &p) { return p.copy_dtype == RS_BF16 ? 2 : p
 static StreamLayout layout_for(const Params &p, int npos) {
     const int NPr = prep_np(npos);
     const bool mma = use_mma(state_bytes(p), NPr);
-    const int nt = NPr <= 2 ? Roles<1, false>::NT : mma ? Roles<8, true>::NT : Roles<8, false>::NT;
+    const int nt = consumer_teams(NPr, mma, p.CC);   // the kernel's Roles<NP, MMA, CC>::NT
     return stream_layout(p.R, (size_t)p.CC * state_bytes(p), p.blk_r, 4 * tile_rec_floats(p.kind, NPr, p.cap, p.CC), nt);
 }
 
@@ -740,7 +754,7 @@ static cudaError_t launch_stream_t(const Params &p, const CUtensorMap &smap, int
     // may start while the prep kernel before it is still running (see grid_dependency_wait)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(Roles<NP, use_mma(TS::bytes, NP)>::THREADS);
+    cfg.blockDim = dim3(Roles<NP, use_mma(TS::bytes, NP), CC>::THREADS);
     cfg.dynamicSmemBytes = lay.total;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
