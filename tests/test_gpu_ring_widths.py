@@ -34,9 +34,9 @@ SHAPES = [
     ("gdn", 32, 128, 1, 4, 3),   # 4 slots
     ("gdn", 24, 64, 1, 16, 5),
     ("gdn", 64, 64, 1, 64, 5),   # 64 slots: sequential sweep in the prep
-    # stages of 64 KB (a 32 KB tile and a 32 KB ring block): three consumer teams instead of four
-    ("gdn", 128, 128, 1, 128, 5),
-    ("m2", 128, 128, 1, 128, 5),
+    # stages of about 68 KB (a 32 KB tile and a 32 KB ring block): three consumer teams instead of four
+    ("gdn", 256, 64, 1, 64, 5),
+    ("m2", 256, 64, 1, 64, 5),
 ]
 # fp32 inputs, fp32 checkpoint without a copy (CUDA-core contraction, sequential sweep)
 SHAPES_F32 = [("m2", 32, 64, 2, 8, 5), ("gdn", 32, 64, 1, 8, 5), ("gdn", 48, 32, 1, 16, 8)]
