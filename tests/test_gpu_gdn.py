@@ -39,7 +39,7 @@ def decode_run(case, sess, steps, K, check_drift=False, errs=None):
 
 
 def test_tiny_gdn_fp32_from_zero(cuda_device):
-    """Test-only mirror of the Mamba-2 config 0: B=2, H=4, dk=dv=16, fp32, K=4, 32 steps."""
+    """The GDN counterpart of the tiny fp32 Mamba-2 case: B=2, H=4, dk=dv=16, fp32, K=4, 32 steps."""
     case = GdnCase(2, 4, 16, 16, rs.RS_F32, seed=100, device=cuda_device, scale=0.5)
     sess = make_session(rs.RS_GDN, 2, 4, 16, 16, cap=4, in_dtype=rs.RS_F32,
                         copy_dtype=rs.RS_NONE, gdn_scale=0.5)

@@ -40,7 +40,7 @@ def decode_run(case, sess, steps, K, check_ptrs=True, check_drift=False, errs=No
 
 
 def test_config0_fp32_from_zero(cuda_device):
-    """Config 0: B=2, H=4, P=N=16, G=1, fp32 throughout, K=4, 32 steps, seed 0."""
+    """The tiny fp32 case: B=2, H=4, P=N=16, G=1, fp32 throughout, K=4, 32 steps, seed 0."""
     case = Mamba2Case(2, 4, 16, 16, 1, rs.RS_F32, seed=0, device=cuda_device)
     sess = make_session(rs.RS_MAMBA2, 2, 4, 16, 16, cap=4, in_dtype=rs.RS_F32,
                         copy_dtype=rs.RS_NONE, A=case.A, D=case.D)

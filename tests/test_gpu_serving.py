@@ -2,13 +2,14 @@
 configuration, on sampled (sequence, head) pairs that the fp64 oracle follows
 one by one: the first and last sequences and heads and a spread in between.
 
-  config 1  Mamba-2 H=80 P=64 N=128, bf16 inputs, fp32 master + bf16 copy, K=8
-  config 2  GDN H=32 dk=dv=128, same precisions, K=8
-  config 3  speculative rounds on both shapes: 5 positions verified per round,
-            Bernoulli(0.7) acceptance, rollback of the rejected suffix, commit
-            once len >= 16, ring of 32
-  config 4  the hybrid stack's layer shapes (Mamba-2 H=128, GDN H=32) with an
-            E4M3 copy and K=16, dual-precision and shared-low-precision arms
+  Mamba-2 decode   H=80 P=64 N=128, bf16 inputs, fp32 master + bf16 copy, K=8
+  GDN decode       H=32 dk=dv=128, same precisions, K=8
+  speculative      rounds on both shapes: 5 positions verified per round,
+                   Bernoulli(0.7) acceptance, rollback of the rejected suffix,
+                   commit once len >= 16, ring of 32
+  E4M3 layers      the hybrid stack's layer shapes (Mamba-2 H=128, GDN H=32)
+                   with an E4M3 copy and K=16, dual-precision and
+                   shared-low-precision arms
 
 Each starts from a 512-step eager fp32 prefill loaded as the checkpoint (the
 oracle runs its own fp64 prefill on the same inputs)."""
@@ -131,7 +132,7 @@ def test_speculative_rounds_at_serving_shape(cuda_device, kind):
 
 @pytest.mark.parametrize("kind", ["m2", "gdn"])
 def test_fp8_copy_layer_shapes_dual_and_shared(cuda_device, kind):
-    """Config 4's layer shapes: errors of both arms at decode steps 1 and 64 on
+    """The hybrid stack's E4M3 layer shapes: errors of both arms at decode steps 1 and 64 on
     the sampled pairs; each arm matches the oracle fed its own quantised
     checkpoint, and the dual arm meets the E4M3 tolerance."""
     K, cap, steps = 16, 16, 64
