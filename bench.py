@@ -10,6 +10,12 @@ steps.
 
 Prints one JSON line.  `--impl reference` times the fp64 CPU oracle instead
 (the reference arm: there is no runnable reference implementation).
+
+`--k-sweep` (one GPU) measures the commit-interval trade-off instead: for
+K = 4, 8, 16, 32 (ring capacity K) the same decode steps with the whole batch
+committing every K-th step, and with staggered commits (sequence b commits at
+the steps i with i = b mod K, through the commit mask), one JSON line per K
+with throughput, per-step time percentiles and state bytes per token.
 """
 import argparse
 import json
@@ -45,6 +51,7 @@ def parse():
     ap.add_argument("--prefill", type=int, default=PREFILL)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-work", type=float, default=20.0)
+    ap.add_argument("--k-sweep", action="store_true")
     return ap.parse_args()
 
 
@@ -428,8 +435,80 @@ def gpu_arm(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------ commit-interval sweep ----
+
+def k_sweep(args):
+    """Replay cost against checkpoint traffic as K varies.  A larger K moves
+    fewer checkpoint bytes per token (10 / K B per state element for the
+    commit) but buffers more entries: the prep reduces up to K entries per
+    head and the streaming pass stages each tile's whole ring block
+    (cap x P x 2 B).  Synchronous commits make every K-th step long;
+    staggered ones spread the same work over all steps."""
+    import torch
+
+    import rs_decode_outputs_b200 as rs
+    from rs_decode_outputs_b200 import inputs as gen
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    A, D, dtb = gen.mamba2_params(H, 1, dev)
+    src = gen.Mamba2Stream(B, H, P, N, G, torch.bfloat16, dtb, 10_001, dev)
+    pool = src.next(64)
+    steps_in = [rs.make_inputs({k: v[t:t + 1] for k, v in pool.items()}) for t in range(64)]
+    nsteps = max(256, args.steps // 8)
+    for K in (4, 8, 16, 32):
+        cfg = rs.make_config(rs.RS_MAMBA2, B, H, P, N, G, cap=K, npos_max=1, in_dtype=rs.RS_BF16,
+                             copy_dtype=rs.RS_BF16, out_dtype=rs.RS_BF16)
+        sess = rs.ReplaySSM(cfg, A=A, D=D, device=dev)
+        g = torch.Generator(device=dev).manual_seed(K)
+        sess.load_checkpoint(0.1 * torch.randn(B, H, P, N, device=dev, generator=g))
+        h, y = sess.handle, sess.new_out()
+        masks = [(torch.arange(B, device=dev) % K == ph).to(torch.int32) for ph in range(K)]
+        res = {}
+        for mode in ("sync", "staggered"):
+            def step(i):
+                rs.rs_decode_step(h, steps_in[i % 64], 1, y)
+                if mode == "sync" and (i + 1) % K == 0:
+                    rs.rs_commit(h, K)
+                elif mode == "staggered":
+                    rs.rs_commit(h, 1, masks[i % K])
+            i = 0
+            for _ in range(4 * K):   # warm-up; staggered lengths settle within K steps
+                step(i)
+                i += 1
+            while i % K:
+                step(i)
+                i += 1
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(nsteps + 1)]
+            torch.cuda.synchronize()
+            ev[0].record(stream)
+            for j in range(nsteps):
+                step(i)
+                i += 1
+                ev[j + 1].record(stream)
+            torch.cuda.synchronize()
+            per = sorted(ev[j].elapsed_time(ev[j + 1]) * 1e3 for j in range(nsteps))
+            total_us = ev[0].elapsed_time(ev[nsteps]) * 1e3
+            res[mode] = {"tokens_per_s": B * nsteps / (total_us * 1e-6), "us_per_step": total_us / nsteps,
+                         "p50_us": per[nsteps // 2], "p99_us": per[min(nsteps - 1, int(0.99 * nsteps))],
+                         "max_us": per[-1]}
+        status, flags = sess.get_error()
+        if status != rs.RS_OK:
+            raise RuntimeError(f"device error flags set at K={K}: {set(flags.tolist())}")
+        line = {"k_sweep": True, "workload": WORKLOAD.replace("K8", f"K{K}"), "commit_interval": K, "ring_cap": K,
+                "steps": nsteps, "state_bytes_per_token": H * P * N * (2 + 10 / K),
+                "ring_block_bytes_per_tile": K * P * 2, **res}
+        print(json.dumps(line), flush=True)
+        del sess
+        torch.cuda.empty_cache()
+
+
 def main():
     args = parse()
+    if args.k_sweep:
+        k_sweep(args)
+        return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if args.impl == "reference":
