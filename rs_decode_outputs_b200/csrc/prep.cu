@@ -413,11 +413,12 @@ m2_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
 
 // -------------------------------------------------------------------- GDN --
 // One warp per (sequence, head); a CTA holds kPrepWarps heads of one sequence.
-// Per-warp shared memory (entries compact, buffer index i at row i):
-//   kraw [cap][CC] | qraw [NP][CC] | alpha [cap] | beta [cap]
+// Per-warp shared memory (entries compact, buffer index i at row i; rows of
+// CC inputs at a pitch of kpitch bytes):
+//   kraw [cap][kpitch] | qraw [NP][kpitch] | alpha [cap] | beta [cap]
 //   (Gram form only:) G, upper triangle by columns [cap (cap - 1) / 2] | P [NP][32]
 struct GdnPrepSmem {
-    size_t k, q, alpha, beta, g, pc, per_warp;
+    size_t k, q, alpha, beta, g, pc, per_warp, kpitch;
 };
 
 // Several positions over bf16 inputs with at most 32 buffered entries take
@@ -428,9 +429,13 @@ __host__ __device__ inline bool gdn_gram(int cap, int CC, int NP, int ib) {
 
 __host__ __device__ inline GdnPrepSmem gdn_prep_smem(int cap, int CC, int NP, int ib) {
     GdnPrepSmem s;
+    // the Gram form reads 8 rows at one column with ldmatrix: rows 16 bytes
+    // apart in the bank pattern (a pitch of 16 mod 128) keep those reads free
+    // of bank conflicts
+    s.kpitch = (size_t)CC * ib + (gdn_gram(cap, CC, NP, ib) ? 16 : 0);
     size_t w = 0;
-    s.k = w;     w = align_up(w + (size_t)cap * CC * ib, 16);
-    s.q = w;     w = align_up(w + (size_t)NP * CC * ib, 16);
+    s.k = w;     w = align_up(w + (size_t)cap * s.kpitch, 16);
+    s.q = w;     w = align_up(w + (size_t)NP * s.kpitch, 16);
     s.alpha = w; w = align_up(w + 4 * (size_t)cap, 16);
     s.beta = w;  w = align_up(w + 4 * (size_t)cap, 16);
     s.g = s.pc = w;
@@ -457,9 +462,10 @@ __host__ __device__ inline GdnPrepSmem gdn_prep_smem(int cap, int CC, int NP, in
 //      in lockstep (one broadcast per position and step);
 //   3. E_j(l) by a suffix-product scan over the lanes, then
 //      coef_j[i] = scale h_i E_j(i + 1)  and  vec_j = E_j(0) (q_j - sum_m h_m k_m).
-// Requires L <= 32, CC a multiple of 16, 1 <= npos <= NP <= 8, npos <= L.
+// Requires L <= 32, CC a multiple of 16, 1 <= npos <= NP <= 8, npos <= L;
+// kraw and qraw rows (bf16) kp bytes apart, kp a multiple of 16.
 template <int CC, int NP>
-__device__ __forceinline__ void gdn_gram_records(const unsigned char *kraw, const unsigned char *qraw,
+__device__ __forceinline__ void gdn_gram_records(const unsigned char *kraw, const unsigned char *qraw, size_t kp,
                                                  const float *alpha, const float *beta, float *gs, float *ps,
                                                  int L, int npos, int lane, float sc, float *coef, int cstr,
                                                  float *vec) {
@@ -478,9 +484,9 @@ __device__ __forceinline__ void gdn_gram_records(const unsigned char *kraw, cons
             for (int nt = 0; nt < 4; ++nt) gacc[mt][nt][f] = 0.f;
         }
     }
-    const unsigned char *arow[2] = {kraw + (size_t)min(lane & 15, L - 1) * CC * 2,
-                                    kraw + (size_t)min(16 + (lane & 15), L - 1) * CC * 2};
-    const unsigned char *qrow = qraw + (size_t)min(lane & 7, npos - 1) * CC * 2;
+    const unsigned char *arow[2] = {kraw + (size_t)min(lane & 15, L - 1) * kp,
+                                    kraw + (size_t)min(16 + (lane & 15), L - 1) * kp};
+    const unsigned char *qrow = qraw + (size_t)min(lane & 7, npos - 1) * kp;
     const int acol = (lane >> 4) * 16, qcol = ((lane >> 3) & 1) * 16;   // bytes
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
@@ -579,14 +585,14 @@ __device__ __forceinline__ void gdn_gram_records(const unsigned char *kraw, cons
 #pragma unroll
         for (int u = 0; u < UPL; ++u) {
             const int c = lane + 32 * u;
-            va[j][u] = (j < npos && c < CC) ? lds_in(qraw, (size_t)j * CC + c, RS_BF16) : 0.f;
+            va[j][u] = (j < npos && c < CC) ? lds_in(qraw + (size_t)j * kp, c, RS_BF16) : 0.f;
         }
     for (int m = 0; m < L; ++m) {
         float kr[UPL];
 #pragma unroll
         for (int u = 0; u < UPL; ++u) {
             const int c = lane + 32 * u;
-            kr[u] = c < CC ? lds_in(kraw, (size_t)m * CC + c, RS_BF16) : 0.f;
+            kr[u] = c < CC ? lds_in(kraw + (size_t)m * kp, c, RS_BF16) : 0.f;
         }
 #pragma unroll
         for (int j = 0; j < NP; ++j) {
@@ -676,10 +682,10 @@ gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
     }
     if (has_head) {
         // ---- one round of asynchronous copies
-        for (int i = 0; i < L; ++i) stage_row(kraw + (size_t)i * rowC, src_row(kblk, in.k, rowC, i), (int)rowC, lane, 32);
+        for (int i = 0; i < L; ++i) stage_row(kraw + i * S.kpitch, src_row(kblk, in.k, rowC, i), (int)rowC, lane, 32);
         if (ok)
             for (int j = 0; j < npos; ++j)
-                stage_row(qraw + (size_t)j * rowC, src_row(qblk, in.q, rowC, L - npos + j), (int)rowC, lane, 32);
+                stage_row(qraw + j * S.kpitch, src_row(qblk, in.q, rowC, L - npos + j), (int)rowC, lane, 32);
         for (int i = lane; i < L; i += 32) {
             const size_t at = ((size_t)(i - L_old) * Bn + b) * H + h;
             cp_async4(alpha + i, i < L_old ? ablk + ((head + i) & p.cap_mask) : in.alpha + at);
@@ -694,7 +700,7 @@ gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
             const float sc = p.gdn_scale;
             const float tscale = p.copy_dtype == RS_E4M3 ? p.scale[tile] : 1.f;
             if constexpr (NP >= 2 && CC % 16 == 0)
-                gdn_gram_records<CC, NP>(kraw, qraw, alpha, beta, reinterpret_cast<float *>(wsm + S.g),
+                gdn_gram_records<CC, NP>(kraw, qraw, S.kpitch, alpha, beta, reinterpret_cast<float *>(wsm + S.g),
                                          reinterpret_cast<float *>(wsm + S.pc), L, npos, lane, sc, coef, cstr,
                                          coef + (size_t)NP * cstr);
             if (lane < npos) trec[lane] = sc * tscale;
@@ -765,7 +771,7 @@ gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
             for (int t = 0; t < T; ++t) {
                 const int slot = (tail + t) & p.cap_mask;
                 const size_t at = ((size_t)t * Bn + b) * H + h;
-                copy_row(kblk + (size_t)slot * rowC, kraw + (size_t)(L_old + t) * rowC, (int)rowC, lane, 32);
+                copy_row(kblk + (size_t)slot * rowC, kraw + (L_old + t) * S.kpitch, (int)rowC, lane, 32);
                 if (pre_qv) {
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
@@ -775,7 +781,7 @@ gdn_prep_kernel(const Params p, int npos, int T, rs_inputs in) {
                 } else {
                     // q: the staged row when the outputs covered this entry (T <= npos)
                     const unsigned char *qsrc = ok && T <= npos
-                                                    ? qraw + (size_t)(npos - T + t) * rowC
+                                                    ? qraw + (npos - T + t) * S.kpitch
                                                     : static_cast<const unsigned char *>(in.q) + at * rowC;
                     copy_row(qblk + (size_t)slot * rowC, qsrc, (int)rowC, lane, 32);
                     if (!pre_v)
