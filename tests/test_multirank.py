@@ -68,3 +68,20 @@ def test_reference_arm_does_no_work_off_rank_zero(capsys):
     args = SimpleNamespace(gpus=2, steps=1, warmup=0)
     bench.reference_arm(args, rank=1)
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_prints_the_contract_line_on_rank_zero(capsys):
+    """One timed step of the oracle arm (a few seconds of CPU): one JSON line
+    with the keys the bench contract asks of the reference arm."""
+    import json
+    args = SimpleNamespace(gpus=1, steps=1, warmup=0)
+    bench.reference_arm(args, rank=0)
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
+    assert d["value"] > 0 and d["higher_is_better"] is True and d["steps"] == 1
+    assert d["config"]["workload"] == bench.WORKLOAD
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
